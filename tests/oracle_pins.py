@@ -1,0 +1,450 @@
+"""Independent pins for the fp64 oracle.
+
+Each pin checks the oracle against something other than itself: a closed
+form (identity, box sum, shifted gather, affine field, constant input), a
+brute-force sum over the whole grid of the bilinear kernel
+g(a,b) = max(0, 1-|a-b|) ("用PyTorch实战DCNv1", section 2), PyTorch's own
+bilinear sampler (grid_sample, zero padding), finite differences and the
+adjoint identity for the gradients. The pins are functions of the oracle
+library handle so that the mutation test can rerun them against deliberately
+broken builds of the oracle.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+F32 = np.float32
+
+
+# ---------------------------------------------------------------- helpers
+def base_grid(Ho, Wo, kh, kw, stride, pad, dil):
+    """by[ho, i], bx[wo, j]: regular grid points of the kernel window."""
+    by = np.arange(Ho)[:, None] * stride[0] - pad[0] + np.arange(kh)[None, :] * dil[0]
+    bx = np.arange(Wo)[:, None] * stride[1] - pad[1] + np.arange(kw)[None, :] * dil[1]
+    return by, bx
+
+
+def positions32(off, Ho, Wo, kh, kw, stride, pad, dil, s):
+    """fp32 sampling positions py, px [B,Ho,Wo,G,K]; s must make s*d exact."""
+    by, bx = base_grid(Ho, Wo, kh, kw, stride, pad, dil)
+    K = kh * kw
+    byk = np.repeat(by, kw, axis=1)  # [Ho, K], k = i*kw + j
+    bxk = np.tile(bx, (1, kh))       # [Wo, K]
+    d = off.astype(F32)
+    py = F32(s) * d[..., 1] + byk[None, :, None, None, :].astype(F32)
+    px = F32(s) * d[..., 0] + bxk[None, None, :, None, :].astype(F32)
+    return py.astype(np.float64), px.astype(np.float64)
+
+
+def brute_force_forward(x, off, mask, G, kh, kw, stride, pad, dil, s, softmax):
+    """out = sum_k m_k sum_{every grid q} g(qx,px) g(qy,py) x(q), by full sums."""
+    B, H, W, GC = x.shape
+    C = GC // G
+    Ho, Wo = oracle.out_hw(H, W, kh, kw, *stride, *pad, *dil)
+    py, px = positions32(off, Ho, Wo, kh, kw, stride, pad, dil, s)
+    m = mask.astype(np.float64)
+    if softmax:
+        e = np.exp(m - m.max(-1, keepdims=True))
+        m = e / e.sum(-1, keepdims=True)
+    qy = np.arange(H, dtype=np.float64)
+    qx = np.arange(W, dtype=np.float64)
+    gy = np.maximum(0.0, 1.0 - np.abs(qy - py[..., None]))  # [B,Ho,Wo,G,K,H]
+    gx = np.maximum(0.0, 1.0 - np.abs(qx - px[..., None]))  # [B,Ho,Wo,G,K,W]
+    xg = x.reshape(B, H, W, G, C).astype(np.float64)
+    # sum over k, qy, qx: m * gy * gx * x[b, qy, qx, g, c]
+    out = np.einsum("bhwgk,bhwgky,bhwgkx,byxgc->bhwgc", m, gy, gx, xg, optimize=True)
+    return out.reshape(B, Ho, Wo, GC)
+
+
+def grid_sample_forward(x, off, mask, G, kh, kw, stride, pad, dil, s, softmax):
+    """The same sum with torch's bilinear grid_sample (zeros padding,
+    align_corners=False: pixel centre i sits at normalised (2i+1)/n - 1)."""
+    B, H, W, GC = x.shape
+    C = GC // G
+    Ho, Wo = oracle.out_hw(H, W, kh, kw, *stride, *pad, *dil)
+    py, px = positions32(off, Ho, Wo, kh, kw, stride, pad, dil, s)
+    m = torch.from_numpy(mask.astype(np.float64))
+    if softmax:
+        m = torch.softmax(m, dim=-1)
+    xt = torch.from_numpy(x.astype(np.float64)).reshape(B, H, W, G, C)
+    out = torch.zeros(B, Ho, Wo, G, C, dtype=torch.float64)
+    for g in range(G):
+        xin = xt[:, :, :, g, :].permute(0, 3, 1, 2)  # [B,C,H,W]
+        for k in range(kh * kw):
+            gx = (2.0 * px[:, :, :, g, k] + 1.0) / W - 1.0
+            gy = (2.0 * py[:, :, :, g, k] + 1.0) / H - 1.0
+            grid = torch.from_numpy(np.stack([gx, gy], -1))
+            v = torch.nn.functional.grid_sample(xin, grid, mode="bilinear", padding_mode="zeros",
+                                                align_corners=False)  # [B,C,Ho,Wo]
+            out[:, :, :, g, :] += m[:, :, :, g, k, None] * v.permute(0, 2, 3, 1)
+    return out.reshape(B, Ho, Wo, GC).numpy()
+
+
+def rand_case(seed, B, H, W, G, C, kh, kw, stride, pad, dil, off_std, quant=None):
+    rng = np.random.default_rng(seed)
+    Ho, Wo = oracle.out_hw(H, W, kh, kw, *stride, *pad, *dil)
+    x = rng.standard_normal((B, H, W, G * C))
+    off = rng.standard_normal((B, Ho, Wo, G, kh * kw, 2)) * off_std
+    if quant is not None:
+        # odd multiples of quant/2: fp32-exact positions that never sit on a grid line
+        off = np.round(off / quant) * quant + quant / 2
+    off = off.astype(F32).astype(np.float64)
+    mask = rng.standard_normal((B, Ho, Wo, G, kh * kw))
+    return x, off, mask
+
+
+GEOMS = [
+    # (H, W, kh, kw, stride, pad, dil)
+    (7, 9, 3, 3, (1, 1), (1, 1), (1, 1)),
+    (8, 6, 3, 3, (2, 2), (1, 1), (1, 1)),
+    (9, 8, 3, 3, (1, 1), (2, 2), (2, 2)),
+    (6, 11, 3, 5, (1, 2), (1, 2), (1, 1)),
+    (5, 5, 1, 1, (1, 1), (0, 0), (1, 1)),
+]
+
+
+# ---------------------------------------------------------------- core pins
+def pin_identity(lib):
+    """Zero offsets and a one-hot centre mask reproduce x exactly."""
+    rng = np.random.default_rng(11)
+    for pad, dil in (((1, 1), (1, 1)), ((2, 2), (2, 2))):
+        x = rng.standard_normal((2, 6, 7, 3 * 4))
+        Ho, Wo = oracle.out_hw(6, 7, 3, 3, 1, 1, *pad, *dil)
+        off = np.zeros((2, Ho, Wo, 3, 9, 2))
+        mask = np.zeros((2, Ho, Wo, 3, 9))
+        mask[..., 4] = 1.0
+        out = oracle.dcn_forward(x, off, mask, G=3, pad=pad, dil=dil, lib=lib)
+        assert np.array_equal(out, x), "identity"
+
+
+def pin_box_sum(lib):
+    """Zero offsets, unit masks: zero-padded window sum (integral image)."""
+    rng = np.random.default_rng(12)
+    for (H, W, kh, kw, stride, pad, dil) in GEOMS:
+        G, C = 2, 3
+        x = rng.standard_normal((1, H, W, G * C))
+        Ho, Wo = oracle.out_hw(H, W, kh, kw, *stride, *pad, *dil)
+        off = np.zeros((1, Ho, Wo, G, kh * kw, 2))
+        mask = np.ones((1, Ho, Wo, G, kh * kw))
+        out = oracle.dcn_forward(x, off, mask, G=G, kh=kh, kw=kw, stride=stride, pad=pad, dil=dil, lib=lib)
+        xp = np.zeros((H + 2 * pad[0] + dil[0] * kh, W + 2 * pad[1] + dil[1] * kw, G * C))
+        xp[pad[0]:pad[0] + H, pad[1]:pad[1] + W] = x[0]
+        ref = np.zeros((Ho, Wo, G * C))
+        for i in range(kh):
+            for j in range(kw):
+                ys = i * dil[0]
+                xs = j * dil[1]
+                ref += xp[ys:ys + (Ho - 1) * stride[0] + 1:stride[0], xs:xs + (Wo - 1) * stride[1] + 1:stride[1]]
+        if (kh, kw, stride, dil) == (3, 3, (1, 1), (1, 1)):
+            # second, independent route: summed-area table of the padded map
+            S = np.zeros((xp.shape[0] + 1, xp.shape[1] + 1, G * C))
+            S[1:, 1:] = xp.cumsum(0).cumsum(1)
+            box = S[3:3 + Ho, 3:3 + Wo] - S[:Ho, 3:3 + Wo] - S[3:3 + Ho, :Wo] + S[:Ho, :Wo]
+            assert np.allclose(box, ref, atol=1e-12)
+        assert np.allclose(out[0], ref, rtol=0, atol=1e-12), "box sum"
+
+
+def pin_shifted_gather(lib):
+    """Integer offsets (dx != dy) give exact shifted gathers, zero outside."""
+    rng = np.random.default_rng(13)
+    for (H, W, kh, kw, stride, pad, dil) in GEOMS:
+        G, C, B = 2, 3, 2
+        K = kh * kw
+        x = rng.standard_normal((B, H, W, G * C))
+        Ho, Wo = oracle.out_hw(H, W, kh, kw, *stride, *pad, *dil)
+        off = rng.integers(-3, 4, size=(B, Ho, Wo, G, K, 2)).astype(np.float64)
+        off[..., 0] += 1.0  # keep dx and dy statistically different
+        mask = rng.standard_normal((B, Ho, Wo, G, K))
+        out = oracle.dcn_forward(x, off, mask, G=G, kh=kh, kw=kw, stride=stride, pad=pad, dil=dil, lib=lib)
+        by, bx = base_grid(Ho, Wo, kh, kw, stride, pad, dil)
+        ref = np.zeros((B, Ho, Wo, G, C))
+        xg = x.reshape(B, H, W, G, C)
+        bb, hh, ww, gg, ii, jj = np.meshgrid(np.arange(B), np.arange(Ho), np.arange(Wo), np.arange(G),
+                                             np.arange(kh), np.arange(kw), indexing="ij")
+        kk = ii * kw + jj
+        yy = by[hh, ii] + off[bb, hh, ww, gg, kk, 1].astype(int)
+        xx = bx[ww, jj] + off[bb, hh, ww, gg, kk, 0].astype(int)
+        ok = (yy >= 0) & (yy < H) & (xx >= 0) & (xx < W)
+        vals = np.where(ok[..., None], xg[bb, np.clip(yy, 0, H - 1), np.clip(xx, 0, W - 1), gg], 0.0)
+        ref = (mask[bb, hh, ww, gg, kk][..., None] * vals).sum(axis=(4, 5))
+        assert np.allclose(out.reshape(B, Ho, Wo, G, C), ref, rtol=0, atol=1e-12), "shifted gather"
+
+
+def pin_affine_field(lib):
+    """Bilinear interpolation is exact on x = a + b*y + c*x inside the map."""
+    rng = np.random.default_rng(14)
+    H, W, G, C = 12, 10, 2, 3
+    a, bcoef, ccoef = rng.standard_normal((3, G * C))
+    yy, xx = np.meshgrid(np.arange(H), np.arange(W), indexing="ij")
+    x = (a + bcoef * yy[..., None] + ccoef * xx[..., None])[None]
+    Ho, Wo = H, W
+    off = rng.uniform(-0.9, 0.9, size=(1, Ho, Wo, G, 9, 2))
+    off = np.round(off * 1024) / 1024  # fp32-exact positions
+    mask = rng.standard_normal((1, Ho, Wo, G, 9))
+    out = oracle.dcn_forward(x, off, mask, G=G, lib=lib)
+    py, px = positions32(off, Ho, Wo, 3, 3, (1, 1), (1, 1), (1, 1), 1.0)
+    inside = ((py >= 0) & (py <= H - 1) & (px >= 0) & (px <= W - 1)).all(axis=(3, 4))
+    field = a.reshape(G, C)[None, None, None, :, None, :] + \
+        bcoef.reshape(G, C)[None, None, None, :, None, :] * py[..., None] + \
+        ccoef.reshape(G, C)[None, None, None, :, None, :] * px[..., None]
+    ref = (mask[..., None] * field).sum(axis=4).reshape(1, Ho, Wo, G * C)
+    assert inside.sum() > 20
+    assert np.allclose(out[inside], ref[inside], rtol=0, atol=1e-11), "affine field"
+
+
+def pin_softmax_constant(lib):
+    """Softmax modulation of a constant map returns the constant inside it."""
+    rng = np.random.default_rng(15)
+    H, W, G, C = 10, 9, 3, 2
+    kappa = 1.75
+    x = np.full((1, H, W, G * C), kappa)
+    off = rng.uniform(-0.45, 0.45, size=(1, H, W, G, 9, 2))
+    mask = rng.standard_normal((1, H, W, G, 9)) * 3.0
+    out = oracle.dcn_forward(x, off, mask, G=G, softmax=True, lib=lib)
+    py, px = positions32(off, H, W, 3, 3, (1, 1), (1, 1), (1, 1), 1.0)
+    inside = ((py >= 0) & (py <= H - 1) & (px >= 0) & (px <= W - 1)).all(axis=(3, 4))
+    assert inside.sum() > 10
+    assert np.allclose(out[inside], kappa, rtol=0, atol=1e-13), "softmax constant"
+    # border pixels, whose taps leave the map, lose part of the unit weight
+    assert (out[~inside] <= kappa + 1e-13).all() and out[~inside].mean() < 0.95 * kappa
+
+
+def pin_softmax_vs_raw(lib):
+    """Softmax mode equals raw mode fed with scipy's softmax over K."""
+    from scipy.special import softmax
+
+    x, off, mask = rand_case(16, 2, 7, 8, 3, 4, 3, 3, (1, 1), (1, 1), (1, 1), 2.0)
+    a = oracle.dcn_forward(x, off, mask, G=3, softmax=True, lib=lib)
+    b = oracle.dcn_forward(x, off, softmax(mask, axis=-1), G=3, softmax=False, lib=lib)
+    assert np.allclose(a, b, rtol=0, atol=1e-13), "softmax vs raw"
+
+
+def pin_brute_force(lib):
+    """The four-corner sum equals the sum over every grid point (random
+    fractional offsets, out-of-range taps included), and matches grid_sample."""
+    for n, (H, W, kh, kw, stride, pad, dil) in enumerate(GEOMS):
+        for s, softmax in ((1.0, False), (0.5, True)):
+            x, off, mask = rand_case(20 + n, 2, H, W, 2, 3, kh, kw, stride, pad, dil, 2.5)
+            out = oracle.dcn_forward(x, off, mask, G=2, kh=kh, kw=kw, stride=stride, pad=pad, dil=dil,
+                                     offset_scale=s, softmax=softmax, lib=lib)
+            ref = brute_force_forward(x, off, mask, 2, kh, kw, stride, pad, dil, s, softmax)
+            assert np.allclose(out, ref, rtol=0, atol=1e-12), "brute force"
+            gs = grid_sample_forward(x, off, mask, 2, kh, kw, stride, pad, dil, s, softmax)
+            assert np.allclose(out, gs, rtol=0, atol=1e-10), "grid_sample"
+
+
+# ---------------------------------------------------------------- backward pins
+def _loss(lib, x, off, mask, go, G, geom, s, softmax):
+    H, W, kh, kw, stride, pad, dil = geom
+    out = oracle.dcn_forward(x, off, mask, G=G, kh=kh, kw=kw, stride=stride, pad=pad, dil=dil,
+                             offset_scale=s, softmax=softmax, lib=lib)
+    return float((go * out).sum())
+
+
+def pin_backward_fd(lib):
+    """Finite differences of <grad_out, out> for the offset and the mask, and
+    the adjoint identity <grad_out, F(x')> = <grad_x, x'> (out is linear in x)."""
+    for softmax in (False, True):
+        geom = (6, 7, 3, 3, (1, 1), (1, 1), (1, 1))
+        H, W, kh, kw, stride, pad, dil = geom
+        G, C = 2, 4
+        # offsets on a 2^-12 lattice keep base + d + h exact in fp32
+        x, off, mask = rand_case(31, 1, H, W, G, C, kh, kw, stride, pad, dil, 1.5, quant=2.0 ** -12)
+        rng = np.random.default_rng(32)
+        Ho, Wo = oracle.out_hw(H, W, kh, kw, *stride, *pad, *dil)
+        go = rng.standard_normal((1, Ho, Wo, G * C))
+        s = 0.5
+        gr = oracle.dcn_backward(x, off, mask, go, G=G, offset_scale=s, softmax=softmax, lib=lib)
+        py, px = positions32(off, Ho, Wo, kh, kw, stride, pad, dil, s)
+        h = 2.0 ** -10
+        checked = 0
+        for idx in map(tuple, rng.integers([0, 0, 0, 0, 0], [1, Ho, Wo, G, 9], size=(40, 5))):
+            for comp, pos in ((0, px[idx]), (1, py[idx])):
+                frac = pos - np.floor(pos)
+                if frac < 4 * h * s or frac > 1 - 4 * h * s:
+                    continue  # the derivative jumps on grid lines
+                op, om = off.copy(), off.copy()
+                op[idx + (comp,)] += h
+                om[idx + (comp,)] -= h
+                fd = (_loss(lib, x, op, mask, go, G, geom, s, softmax)
+                      - _loss(lib, x, om, mask, go, G, geom, s, softmax)) / (2 * h)
+                assert abs(fd - gr["grad_offset"][idx + (comp,)]) < 1e-9 * (1 + abs(fd)), "fd offset"
+                checked += 1
+            hm = 1e-6
+            mp, mm = mask.copy(), mask.copy()
+            mp[idx] += hm
+            mm[idx] -= hm
+            fd = (_loss(lib, x, off, mp, go, G, geom, s, softmax)
+                  - _loss(lib, x, off, mm, go, G, geom, s, softmax)) / (2 * hm)
+            assert abs(fd - gr["grad_mask"][idx]) < 1e-7 * (1 + abs(fd)), "fd mask"
+        assert checked > 40
+        # adjoint identity for grad_x, and each unit vector for a handful of entries
+        xp = rng.standard_normal(x.shape)
+        lhs = _loss(lib, xp, off, mask, go, G, geom, s, softmax)
+        rhs = float((gr["grad_x"] * xp).sum())
+        assert abs(lhs - rhs) < 1e-10 * (1 + abs(lhs)), "adjoint grad_x"
+        for flat in rng.integers(0, x.size, size=8):
+            e = np.zeros(x.size)
+            e[flat] = 1.0
+            v = _loss(lib, e.reshape(x.shape), off, mask, go, G, geom, s, softmax)
+            assert abs(v - gr["grad_x"].reshape(-1)[flat]) < 1e-12, "unit grad_x"
+
+
+def pin_backward_autograd(lib):
+    """The offset and mask gradients agree with torch.autograd through the
+    grid_sample formulation (a third, library route)."""
+    geom = (5, 6, 3, 3, (1, 1), (1, 1), (1, 1))
+    H, W, kh, kw, stride, pad, dil = geom
+    G, C = 2, 3
+    x, off, mask = rand_case(41, 1, H, W, G, C, kh, kw, stride, pad, dil, 1.2, quant=2.0 ** -12)
+    rng = np.random.default_rng(42)
+    go = rng.standard_normal((1, H, W, G * C))
+    gr = oracle.dcn_backward(x, off, mask, go, G=G, lib=lib)
+    by, bx = base_grid(H, W, kh, kw, stride, pad, dil)
+    byk = torch.from_numpy(np.repeat(by, kw, axis=1).astype(np.float64))
+    bxk = torch.from_numpy(np.tile(bx, (1, kh)).astype(np.float64))
+    offt = torch.from_numpy(off).requires_grad_(True)
+    mt = torch.from_numpy(mask).requires_grad_(True)
+    xt = torch.from_numpy(x).requires_grad_(True)
+    out = torch.zeros(1, H, W, G, C, dtype=torch.float64)
+    for g in range(G):
+        xin = xt.reshape(1, H, W, G, C)[:, :, :, g, :].permute(0, 3, 1, 2)
+        for k in range(9):
+            px = bxk[None, None, :, k] + offt[:, :, :, g, k, 0]
+            py = byk[None, :, None, k] + offt[:, :, :, g, k, 1]
+            grid = torch.stack([(2 * px + 1) / W - 1, (2 * py + 1) / H - 1], -1)
+            v = torch.nn.functional.grid_sample(xin, grid, mode="bilinear", padding_mode="zeros",
+                                                align_corners=False)
+            out[:, :, :, g, :] = out[:, :, :, g, :] + mt[:, :, :, g, k, None] * v.permute(0, 2, 3, 1)
+    (out.reshape(1, H, W, G * C) * torch.from_numpy(go)).sum().backward()
+    assert np.allclose(gr["grad_offset"], offt.grad.numpy(), rtol=0, atol=1e-9), "autograd offset"
+    assert np.allclose(gr["grad_mask"], mt.grad.numpy(), rtol=0, atol=1e-10), "autograd mask"
+    assert np.allclose(gr["grad_x"], xt.grad.numpy(), rtol=0, atol=1e-10), "autograd x"
+
+
+# ---------------------------------------------------------------- aggregation pins
+def agg_case(seed, B=1, cams=2, scales=((5, 7), (3, 4)), A=3, P=2, G=2, C=3, lo=-0.1, hi=1.1, quant=None):
+    rng = np.random.default_rng(seed)
+    hw = sum(h * w for h, w in scales)
+    rows = cams * hw
+    feat = rng.standard_normal((B, rows, G * C))
+    shape = np.array([[list(s) for s in scales]] * cams, dtype=np.int32)
+    start = np.array([[c * hw + sum(h * w for h, w in scales[:s]) for s in range(len(scales))]
+                      for c in range(cams)], dtype=np.int32)
+    loc = rng.uniform(lo, hi, size=(B, A, P, cams, 2))
+    if quant is not None:
+        loc = np.round(loc / quant) * quant
+    loc = loc.astype(F32)
+    w = rng.standard_normal((B, A, P, cams, len(scales), G))
+    return feat, shape, start, loc, w
+
+
+def agg_pos32(u, n):
+    """fp32 position u*n - 0.5 with one rounding (the product and the shift
+    are exact in fp64 for a 24-bit u and a small integer n)."""
+    return (u.astype(np.float64) * n - 0.5).astype(F32).astype(np.float64)
+
+
+def agg_brute_force(feat, shape, start, loc, w):
+    """Explicit per-camera, per-scale maps and a sum over every grid point."""
+    B, rows, GC = feat.shape
+    _, A, P, cams, S, G = w.shape
+    C = GC // G
+    out = np.zeros((B, A, G, C))
+    for b in range(B):
+        for cam in range(cams):
+            for s in range(S):
+                Hs, Ws = int(shape[cam, s, 0]), int(shape[cam, s, 1])
+                r0 = int(start[cam, s])
+                fmap = feat[b, r0:r0 + Hs * Ws].reshape(Hs, Ws, G, C)
+                px = agg_pos32(loc[b, :, :, cam, 0], Ws)  # [A,P]
+                py = agg_pos32(loc[b, :, :, cam, 1], Hs)
+                gy = np.maximum(0, 1 - np.abs(np.arange(Hs) - py[..., None]))
+                gx = np.maximum(0, 1 - np.abs(np.arange(Ws) - px[..., None]))
+                out[b] += np.einsum("apg,apy,apx,yxgc->agc", w[b, :, :, cam, s, :], gy, gx, fmap)
+    return out.reshape(B, A, GC)
+
+
+def pin_agg_brute_force(lib):
+    for seed in range(3):
+        feat, shape, start, loc, w = agg_case(50 + seed)
+        out = oracle.agg_forward(feat, shape, start, loc, w, lib=lib)
+        ref = agg_brute_force(feat, shape, start, loc, w)
+        assert np.allclose(out, ref, rtol=0, atol=1e-12), "agg brute force"
+
+
+def pin_agg_grid_sample(lib):
+    feat, shape, start, loc, w = agg_case(60, cams=3, scales=((6, 9), (4, 5), (2, 3)), A=4, P=3)
+    out = oracle.agg_forward(feat, shape, start, loc, w, lib=lib)
+    B, rows, GC = feat.shape
+    _, A, P, cams, S, G = w.shape
+    C = GC // G
+    ref = torch.zeros(B, A, G, C, dtype=torch.float64)
+    for cam in range(cams):
+        for s in range(S):
+            Hs, Ws = int(shape[cam, s, 0]), int(shape[cam, s, 1])
+            r0 = int(start[cam, s])
+            fm = torch.from_numpy(feat[:, r0:r0 + Hs * Ws]).reshape(B, Hs, Ws, G, C)
+            px = torch.from_numpy(agg_pos32(loc[:, :, :, cam, 0], Ws))
+            py = torch.from_numpy(agg_pos32(loc[:, :, :, cam, 1], Hs))
+            grid = torch.stack([(2 * px + 1) / Ws - 1, (2 * py + 1) / Hs - 1], -1)  # [B,A,P,2]
+            for g in range(G):
+                v = torch.nn.functional.grid_sample(fm[..., g, :].permute(0, 3, 1, 2), grid,
+                                                    mode="bilinear", padding_mode="zeros",
+                                                    align_corners=False)  # [B,C,A,P]
+                ref[:, :, g, :] += (torch.from_numpy(w[:, :, :, cam, s, g])[:, None] * v).sum(-1).permute(0, 2, 1)
+    assert np.allclose(out, ref.reshape(B, A, GC).numpy(), rtol=0, atol=1e-10), "agg grid_sample"
+
+
+def pin_agg_backward(lib):
+    """Finite differences (locations on a 2^-14 lattice keep loc*size exact),
+    linearity in the weights, and the adjoint identity for grad_feat."""
+    feat, shape, start, loc, w = agg_case(70, quant=2.0 ** -14)
+    rng = np.random.default_rng(71)
+    B, rows, GC = feat.shape
+    _, A, P, cams, S, G = w.shape
+    go = rng.standard_normal((B, A, GC))
+    gr = oracle.agg_backward(feat, shape, start, loc, w, go, lib=lib)
+
+    def loss(f, l, ww):
+        return float((go * oracle.agg_forward(f, shape, start, l, ww, lib=lib)).sum())
+
+    h = 2.0 ** -12
+    checked = 0
+    for idx in map(tuple, rng.integers([0, 0, 0, 0, 0], [B, A, P, cams, 2], size=(30, 5))):
+        lp, lm = loc.copy(), loc.copy()
+        lp[idx] += F32(h)
+        lm[idx] -= F32(h)
+        # skip when any scale's position crosses a grid line
+        cam, comp = idx[3], idx[4]
+        crosses = False
+        for s in range(S):
+            n = shape[cam, s, 1 - comp]
+            a_ = float(lm[idx]) * n - 0.5
+            b_ = float(lp[idx]) * n - 0.5
+            if np.floor(a_) != np.floor(b_) or a_ == np.floor(a_):
+                crosses = True
+        if crosses:
+            continue
+        fd = (loss(feat, lp, w) - loss(feat, lm, w)) / (2 * h)
+        assert abs(fd - gr["grad_loc"][idx]) < 1e-9 * (1 + abs(fd)), "agg fd loc"
+        checked += 1
+    assert checked > 10
+    for idx in map(tuple, rng.integers([0] * 6, [B, A, P, cams, S, G], size=(12, 6))):
+        wp = w.copy()
+        wp[idx] += 1.0
+        assert abs(loss(feat, loc, wp) - loss(feat, loc, w) - gr["grad_weights"][idx]) < 1e-10, "agg w"
+    fp = rng.standard_normal(feat.shape)
+    lhs = loss(fp, loc, w)
+    rhs = float((gr["grad_feat"] * fp).sum())
+    assert abs(lhs - rhs) < 1e-10 * (1 + abs(lhs)), "agg adjoint"
+
+
+CORE_PINS = [pin_identity, pin_box_sum, pin_shifted_gather, pin_affine_field, pin_softmax_constant,
+             pin_softmax_vs_raw, pin_brute_force]
+BACKWARD_PINS = [pin_backward_fd, pin_backward_autograd]
+AGG_PINS = [pin_agg_brute_force, pin_agg_grid_sample, pin_agg_backward]
+ALL_PINS = CORE_PINS + BACKWARD_PINS + AGG_PINS
