@@ -1,0 +1,481 @@
+"""Benchmark of the deformable sampling core on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-rows] [--no-cpu]
+
+One step = one dcn_core_forward over one batch of the DCNv4 YOLO-P4 workload
+(B=8 per GPU, 40x40, G=16 x C=32, 3x3, fp16 storage, fp32 accumulation, raw
+modulation).  Inputs rotate over enough resident copies to exceed 4x the L2
+size, so every step reads HBM.  The K timed steps are replayed from CUDA
+graphs and bracketed by a barrier and synchronisations; the time is the max
+over ranks of CUDA-event time on the launching stream.  Rank 0 prints one
+JSON line.  Under torchrun each rank runs its own batch (weak scaling, no
+collective on the data path; the only collectives are the barrier and the
+max-over-ranks of the time).
+
+--impl reference times the fp64 CPU oracle (the reference this build is
+checked against) on the host cores, on rank 0, on a bounded sample of the
+same workload; other ranks exit without work.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic_inputs as si  # noqa: E402
+
+METRIC = "deform-sample fwd Gsamples/s & achieved HBM GB/s (% of peak), DCNv4 P4 shape"
+WORKLOAD = ("DCNv4 core forward, YOLO-P4 shape: B=8 per GPU, H=W=40, 512 ch as G=16 x C=32, 3x3, "
+            "stride 1, pad 1, dil 1, raw modulation, fp16 storage / fp32 accumulate; x~N(0,1), "
+            "offsets~N(0,3), mask~N(0,1)")
+FALLBACK_HBM_GBS = 6650.0
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "deformable_convolution_sampling_dcn_b200", "csrc", f)
+                  for f in ("dcn_forward_plane.cu", "dcn_forward_generic.cu", "dcn_common.cuh")]
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """Polls SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clocks_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # NVML unavailable: report no clocks
+            self.ok = False
+        self._period = period_s
+        self._t = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": len(self.samples)}
+        names = [n for n, bit in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def build_sets(shape, seed, dev, l2_bytes):
+    inp = si.core_inputs(shape, seed, offset_std=3.0)
+    x, off, m = (inp[k].to(dev) for k in ("x", "offset", "mask"))
+    out_shape = (shape.B, shape.Ho, shape.Wo, shape.G * shape.C)
+    footprint = shape.compulsory_bytes()
+    R = max(2, math.ceil(4 * l2_bytes / footprint))
+    sets = []
+    for _ in range(R):
+        sets.append((x.clone(), off.clone(), m.clone(), torch.empty(out_shape, dtype=x.dtype, device=dev)))
+    return inp, sets, R, footprint
+
+
+def capture(fn_list, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for fn in fn_list:
+            fn()
+    return g
+
+
+def time_steps(make_call, sets, K, W, stream, barrier, world):
+    """Replay K calls (rotating over `sets`) from CUDA graphs; returns ms (max over ranks)."""
+    R = len(sets)
+    calls = [make_call(s) for s in sets]
+    for c in calls:  # eager warm-up of each set (also validates the launch)
+        c()
+    torch.cuda.synchronize()
+    g_full = capture(calls, stream)
+    rem = K % R
+    g_rem = capture(calls[:rem], stream) if rem else None
+    full = K // R
+    wfull = max(1, math.ceil(W / R))
+    for _ in range(wfull):
+        g_full.replay()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(full):
+            g_full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    del g_full, g_rem
+    return ms
+
+
+def run_ours(args, world, rank, local):
+    import deformable_convolution_sampling_dcn_b200 as dcn
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+
+        def barrier():
+            torch.distributed.barrier()
+    else:
+        def barrier():
+            pass
+
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+    shape = si.DCNV4_P4
+    inp, sets, R, footprint = build_sets(shape, si.SEEDS["dcnv4_p4"] + 1000 * rank, dev, l2)
+    stream = torch.cuda.Stream(dev)
+
+    def make_call(s):
+        x, off, m, out = s
+        return lambda: dcn.dcn_core_forward(x, off, m, group=shape.G, out=out)
+
+    K, W = args.steps, args.warmup
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    with sampler:
+        ms = time_steps(make_call, sets, K, W, stream, barrier, world)
+    clocks = sampler.summary()
+    step_s = ms / 1e3 / K
+    samples_all = shape.samples * world
+    value = samples_all / step_s / 1e9  # Gsamples/s, whole job
+    bytes_per_launch = shape.compulsory_bytes()
+    achieved = bytes_per_launch / step_s / 1e9
+    peak, peak_kind = peaks()
+    traffic = None
+    if os.path.exists(TRAFFIC_FILE):
+        with open(TRAFFIC_FILE) as f:
+            tr = json.load(f)
+        ent = tr.get("dcnv4_p4_forward")
+        if ent and ent.get("kernel_hash") == kernel_hash():
+            traffic = ent["dram_bytes_per_launch"]
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    e2e = measure_e2e(dcn, shape, inp, dev, stream, min(K, args.e2e_steps), barrier, world)
+
+    rows = measure_rows(dcn, dev, stream, l2, barrier, world) if (args.rows and world == 1) else None
+
+    cpu = None
+    if rank == 0 and world == 1 and args.cpu:
+        cpu = cpu_baseline(args.cpu_seconds)
+
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "Gsamples/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": round(ms / K, 6), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B_per_gpu": shape.B, "global_batch": shape.B * world,
+                       "H": shape.H, "W": shape.W, "G": shape.G, "C": shape.C, "kernel": [3, 3],
+                       "storage": "f16", "accumulate": "f32",
+                       "samples_per_step_per_gpu": shape.samples,
+                       "l2": f"{R} rotating resident input sets ({R * footprint / 1e6:.0f} MB) > 4x L2 "
+                             f"({l2 / 1e6:.0f} MB); no flush",
+                       "timing": "CUDA graphs of the rotating launches, CUDA events on the launching stream",
+                       "parallelism": f"batch shard x{world}, no data-path collective" if world > 1 else "1 GPU"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                         else "fallback 6.65 TB/s",
+                         "algorithmic_bytes_per_launch": bytes_per_launch,
+                         "kernel": "dcn_core_forward (one launch per step)"},
+            "clocks": clocks,
+            "e2e": e2e,
+            "gpu_launches": K,
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        if rows is not None:
+            line["rows"] = rows
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def measure_e2e(dcn, shape, inp, dev, stream, E, barrier, world):
+    """Same metric through dcn_core_forward with host buffers: pinned H2D of
+    the step's inputs, the call, D2H of the output, all inside the timed region."""
+    hx, hoff, hm = (inp[k].pin_memory() for k in ("x", "offset", "mask"))
+    hout = torch.empty((shape.B, shape.Ho, shape.Wo, shape.G * shape.C), dtype=hx.dtype).pin_memory()
+    dx, doff, dm = (torch.empty_like(t, device=dev) for t in (hx, hoff, hm))
+    dout = torch.empty(hout.shape, dtype=hx.dtype, device=dev)
+    E = max(1, E)
+
+    def step():
+        dx.copy_(hx, non_blocking=True)
+        doff.copy_(hoff, non_blocking=True)
+        dm.copy_(hm, non_blocking=True)
+        dcn.dcn_core_forward(dx, doff, dm, group=shape.G, out=dout)
+        hout.copy_(dout, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(E):
+            step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = sum(t.numel() * t.element_size() for t in (hx, hoff, hm))
+    d2h = hout.numel() * hout.element_size()
+    return {"value": round(shape.samples * world / (ms / 1e3 / E) / 1e9, 3), "unit": "Gsamples/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": E,
+            "ms_per_step": round(ms / E, 4)}
+
+
+def measure_rows(dcn, dev, stream, l2, barrier, world, steps=280):
+    """Per-workload device times of every hot-path row (context for the headline)."""
+    out = {}
+
+    def core_fwd(name):
+        shape, inp = si.workload_core(name)
+        x, off, m = (inp[k].to(dev) for k in ("x", "offset", "mask"))
+        R = max(2, math.ceil(4 * l2 / shape.compulsory_bytes()))
+        sets = [(x.clone(), off.clone(), m.clone(),
+                 torch.empty((shape.B, shape.Ho, shape.Wo, shape.G * shape.C), dtype=x.dtype, device=dev))
+                for _ in range(R)]
+        cfg = dict(group=shape.G, kernel=(shape.kh, shape.kw), stride=(shape.stride_h, shape.stride_w),
+                   pad=(shape.pad_h, shape.pad_w), dil=(shape.dil_h, shape.dil_w), softmax=shape.softmax)
+
+        def mk(s):
+            return lambda: dcn.dcn_core_forward(s[0], s[1], s[2], out=s[3], **cfg)
+
+        ms = time_steps(mk, sets, steps, 3 * R, stream, barrier, world) / steps
+        out[name] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(shape.samples / ms / 1e6, 2),
+                     "GB_s": round(shape.compulsory_bytes() / ms / 1e6, 1), "R": R}
+        del sets
+
+    for n in ("dcnv3_tiny", "dcnv3_p3", "dcnv3_p3_dil2"):
+        core_fwd(n)
+
+    # DCNv4 backward at the P4 shape, fp32
+    shape, inp = si.workload_core("dcnv4_p4_bwd")
+    t = [inp[k].to(dev) for k in ("x", "offset", "mask", "grad_out")]
+    R = max(2, math.ceil(4 * l2 / shape.compulsory_bytes(backward=True)))
+    sets = [[u.clone() for u in t] + [torch.empty_like(t[0]), torch.empty_like(t[1]), torch.empty_like(t[2])]
+            for _ in range(R)]
+
+    def mkb(s):
+        return lambda: dcn.dcn_core_backward(s[0], s[1], s[2], s[3], group=shape.G, grad_x=s[4],
+                                             grad_offset=s[5], grad_mask=s[6])
+
+    ms = time_steps(mkb, sets, steps, 3 * R, stream, barrier, world) / steps
+    out["dcnv4_p4_bwd"] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(shape.samples / ms / 1e6, 2),
+                           "GB_s": round(shape.compulsory_bytes(backward=True) / ms / 1e6, 1), "R": R}
+    del sets
+
+    # Sparse4D aggregation forward
+    a = si.SPARSE4D
+    inp = si.agg_inputs(a, si.SEEDS["sparse4d"])
+    keys = ("feat", "spatial_shape", "scale_start_index", "sampling_location", "weights")
+    t = [inp[k].to(dev) for k in keys]
+    R = max(2, math.ceil(4 * l2 / a.compulsory_bytes()))
+    sets = [[u.clone() for u in t] + [torch.empty((a.B, a.num_anchors, a.G * a.C), device=dev)] for _ in range(R)]
+
+    def mka(s):
+        return lambda: dcn.deform_agg_forward(*s[:5], out=s[5])
+
+    ms = time_steps(mka, sets, steps, 3 * R, stream, barrier, world) / steps
+    out["sparse4d"] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(a.samples / ms / 1e6, 2),
+                       "GB_s": round(a.compulsory_bytes() / ms / 1e6, 1), "R": R}
+    return out
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(seconds: float):
+    """The fp64 oracle as it stands on all host cores: whole DCNv4-P4 batches,
+    repeated until `seconds` of wall time have passed (at least once)."""
+    import oracle
+
+    n = oracle.set_threads(cpu_threads())
+    shape, inp = si.workload_core("dcnv4_p4")
+    x, off, m = (inp[k].double().numpy() for k in ("x", "offset", "mask"))
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.dcn_forward(x, off, m, G=shape.G)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": round(shape.samples * reps / el / 1e9, 5), "unit": "Gsamples/s", "cores": n,
+            "kind": "oracle",
+            "sample": f"{reps} whole DCNv4-P4 batches (B=8, {shape.samples} samples each) in {el:.1f} s, "
+                      f"fp64 C loops, OpenMP over (b, output row)"}
+
+
+def run_reference(args, world, rank):
+    """The oracle as it stands, on the host cores, one bounded sample per step.
+
+    Groups are independent, so a step runs the oracle on `ng` whole groups of
+    one image (every output pixel and tap of those groups), sized so that the
+    W + K steps take about a minute."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+
+    n = oracle.set_threads(cpu_threads())
+    shape, inp = si.workload_core("dcnv4_p4")
+    x, off, m = (inp[k].double().numpy() for k in ("x", "offset", "mask"))
+    C, G = shape.C, shape.G
+
+    def group_slice(b, g0, ng):
+        return (np.ascontiguousarray(x[b:b + 1, :, :, g0 * C:(g0 + ng) * C]),
+                np.ascontiguousarray(off[b:b + 1, :, :, g0:g0 + ng]),
+                np.ascontiguousarray(m[b:b + 1, :, :, g0:g0 + ng]))
+
+    t0 = time.perf_counter()
+    xs, os_, ms_ = group_slice(0, 0, 1)
+    for _ in range(3):
+        oracle.dcn_forward(xs, os_, ms_, G=1)
+    per_group = (time.perf_counter() - t0) / 3
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    ng = int(max(1, min(G, budget / max(per_group, 1e-9))))
+    slices = [group_slice(b, g0, ng) for b in range(shape.B) for g0 in range(0, G - ng + 1, ng)]
+
+    def step(i):
+        xs, os_, ms_ = slices[i % len(slices)]
+        oracle.dcn_forward(xs, os_, ms_, G=ng)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    el = time.perf_counter() - t0
+    per_step_samples = shape.Ho * shape.Wo * ng * shape.K
+    v = per_step_samples * args.steps / el / 1e9
+    sample = (f"each step: {ng} of {G} groups of one DCNv4-P4 image, all {shape.Ho}x{shape.Wo} pixels and "
+              f"{shape.K} taps ({per_step_samples} samples); fp64 C oracle, OpenMP")
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "Gsamples/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B_per_gpu": shape.B, "global_batch": shape.B,
+                       "parallelism": "host cores"},
+            "cpu_baseline": {"value": round(v, 6), "unit": "Gsamples/s", "cores": n, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(v, 6), "unit": "Gsamples/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=14000)
+    ap.add_argument("--warmup", type=int, default=140)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--no-rows", dest="rows", action="store_false")
+    ap.add_argument("--no-cpu", dest="cpu", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_env()
+    if world != args.gpus and world != 1:
+        print(f"warning: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

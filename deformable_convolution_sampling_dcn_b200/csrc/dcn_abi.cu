@@ -1,0 +1,214 @@
+// C ABI of the library: host-side argument checks, then one launch (or a
+// memset and a launch) on the caller's stream.  No allocation, no
+// synchronisation.  See include/dcn_b200.h for the contract.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/dcn_b200.h"
+#include "dcn_launch.h"
+
+namespace {
+
+thread_local char g_detail[256] = "no error";
+
+dcn_status fail(dcn_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+dcn_status fail(dcn_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+dcn_status cuda_status(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return DCN_OK;
+    return fail(DCN_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+size_t dtype_size(int32_t dt) { return dt == DCN_F32 ? 4 : 2; }
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+const int kMaxDim = 1 << 20;
+
+// Checks shared by the core calls; fills Ho/Wo.
+dcn_status check_core(const dcn_params *p, int *Ho, int *Wo) {
+    if (!p) return fail(DCN_ERR_NULL, "params is NULL");
+    if (p->dtype < DCN_F32 || p->dtype > DCN_BF16) return fail(DCN_ERR_UNSUPPORTED, "dtype %d", p->dtype);
+    if (p->mask_mode != DCN_MASK_RAW && p->mask_mode != DCN_MASK_SOFTMAX)
+        return fail(DCN_ERR_UNSUPPORTED, "mask_mode %d", p->mask_mode);
+    if (p->B < 0 || p->H < 1 || p->W < 1 || p->G < 1 || p->C < 1 || p->kh < 1 || p->kw < 1)
+        return fail(DCN_ERR_SHAPE, "sizes must be positive (B may be 0)");
+    if (p->B > kMaxDim || p->H > kMaxDim || p->W > kMaxDim || p->G > kMaxDim || p->C > kMaxDim ||
+        p->kh > 64 || p->kw > 64)
+        return fail(DCN_ERR_SHAPE, "a size exceeds its limit");
+    if (p->stride_h < 1 || p->stride_w < 1 || p->dil_h < 1 || p->dil_w < 1)
+        return fail(DCN_ERR_SHAPE, "stride and dilation must be >= 1");
+    if (p->pad_h < 0 || p->pad_w < 0 || p->pad_h > kMaxDim || p->pad_w > kMaxDim)
+        return fail(DCN_ERR_SHAPE, "padding must be in [0, 2^20]");
+    if (!isfinite(p->offset_scale)) return fail(DCN_ERR_SHAPE, "offset_scale is not finite");
+    const long long eh = (long long)p->dil_h * (p->kh - 1) + 1, ew = (long long)p->dil_w * (p->kw - 1) + 1;
+    const long long ho = ((long long)p->H + 2LL * p->pad_h - eh), wo = ((long long)p->W + 2LL * p->pad_w - ew);
+    if (ho < 0 || wo < 0) return fail(DCN_ERR_SHAPE, "kernel extent exceeds the padded input");
+    *Ho = (int)(ho / p->stride_h + 1);
+    *Wo = (int)(wo / p->stride_w + 1);
+    const size_t es = dtype_size(p->dtype);
+    const size_t row = (size_t)p->C * es;
+    if (row % 16 != 0 || row / 16 > 16 || ((row / 16) & (row / 16 - 1)) != 0)
+        return fail(DCN_ERR_UNSUPPORTED, "C*sizeof(dtype) = %zu bytes; supported: 16, 32, 64, 128, 256", row);
+    if ((long long)p->G * p->C > kMaxDim) return fail(DCN_ERR_SHAPE, "G*C exceeds 2^20");
+    return DCN_OK;
+}
+
+dcnb::CoreArgs core_args(const dcn_params *p, int Ho, int Wo) {
+    dcnb::CoreArgs a;
+    memset(&a, 0, sizeof(a));
+    a.B = p->B; a.H = p->H; a.W = p->W; a.G = p->G; a.C = p->C; a.kh = p->kh; a.kw = p->kw;
+    a.sh = p->stride_h; a.sw = p->stride_w; a.ph = p->pad_h; a.pw = p->pad_w;
+    a.dh = p->dil_h; a.dw = p->dil_w; a.Ho = Ho; a.Wo = Wo;
+    a.offset_scale = p->offset_scale;
+    a.softmax = p->mask_mode == DCN_MASK_SOFTMAX;
+    a.dtype = (dcnb::DType)p->dtype;
+    return a;
+}
+
+dcn_status check_agg(const dagg_params *p) {
+    if (!p) return fail(DCN_ERR_NULL, "params is NULL");
+    if (p->dtype < DCN_F32 || p->dtype > DCN_BF16) return fail(DCN_ERR_UNSUPPORTED, "dtype %d", p->dtype);
+    if (p->B < 0 || p->num_cams < 1 || p->num_scales < 1 || p->num_rows < 1 || p->num_anchors < 0 ||
+        p->num_pts < 1 || p->G < 1 || p->C < 1)
+        return fail(DCN_ERR_SHAPE, "sizes must be positive (B and num_anchors may be 0)");
+    if ((long long)p->num_cams * p->num_scales > 4096 || (long long)p->num_pts * p->num_cams > (1 << 20) ||
+        (long long)p->G * p->C > kMaxDim)
+        return fail(DCN_ERR_SHAPE, "a size exceeds its limit");
+    const size_t row = (size_t)p->C * dtype_size(p->dtype);
+    if (row % 16 != 0 || row / 16 > 16 || ((row / 16) & (row / 16 - 1)) != 0)
+        return fail(DCN_ERR_UNSUPPORTED, "C*sizeof(dtype) = %zu bytes; supported: 16, 32, 64, 128, 256", row);
+    return DCN_OK;
+}
+
+dcnb::AggArgs agg_args(const dagg_params *p) {
+    dcnb::AggArgs a;
+    memset(&a, 0, sizeof(a));
+    a.B = p->B; a.cams = p->num_cams; a.scales = p->num_scales; a.rows = p->num_rows;
+    a.A = p->num_anchors; a.P = p->num_pts; a.G = p->G; a.C = p->C;
+    a.dtype = (dcnb::DType)p->dtype;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t dcn_abi_version(void) { return DCN_ABI_VERSION; }
+
+const char *dcn_last_error_detail(void) { return g_detail; }
+
+const char *dcn_status_string(dcn_status s) {
+    switch (s) {
+        case DCN_OK: return "DCN_OK";
+        case DCN_ERR_NULL: return "DCN_ERR_NULL: a required pointer is NULL";
+        case DCN_ERR_SHAPE: return "DCN_ERR_SHAPE: invalid sizes";
+        case DCN_ERR_UNSUPPORTED: return "DCN_ERR_UNSUPPORTED: configuration not implemented";
+        case DCN_ERR_ALIGN: return "DCN_ERR_ALIGN: misaligned pointer";
+        case DCN_ERR_CUDA: return "DCN_ERR_CUDA: CUDA runtime error";
+    }
+    return "unknown dcn_status";
+}
+
+dcn_status dcn_core_output_hw(const dcn_params *p, int32_t *Ho, int32_t *Wo) {
+    int ho = 0, wo = 0;
+    const dcn_status s = check_core(p, &ho, &wo);
+    if (s != DCN_OK) return s;
+    if (!Ho || !Wo) return fail(DCN_ERR_NULL, "Ho/Wo output pointer is NULL");
+    *Ho = ho;
+    *Wo = wo;
+    return DCN_OK;
+}
+
+dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offset, const void *mask,
+                            void *out, dcn_stream_t stream) {
+    int Ho, Wo;
+    dcn_status s = check_core(p, &Ho, &Wo);
+    if (s != DCN_OK) return s;
+    if (p->B == 0) return DCN_OK;
+    if (!x || !offset || !mask || !out) return fail(DCN_ERR_NULL, "x, offset, mask and out are required");
+    const size_t es = dtype_size(p->dtype);
+    if (!aligned(x, 16) || !aligned(out, 16)) return fail(DCN_ERR_ALIGN, "x and out must be 16-byte aligned");
+    if (!aligned(offset, 2 * es) || !aligned(mask, es))
+        return fail(DCN_ERR_ALIGN, "offset must be aligned to 2*sizeof(dtype), mask to sizeof(dtype)");
+    dcnb::CoreArgs a = core_args(p, Ho, Wo);
+    a.x = x; a.offset = offset; a.mask = mask; a.out = out;
+    bool handled = false;
+    cudaError_t e = dcnb::launch_core_forward_plane(a, (cudaStream_t)stream, &handled);
+    if (!handled) e = dcnb::launch_core_forward_generic(a, (cudaStream_t)stream);
+    return cuda_status(e, "dcn_core_forward launch");
+}
+
+dcn_status dcn_core_backward(const dcn_params *p, const void *x, const void *offset, const void *mask,
+                             const void *grad_out, void *grad_x, void *grad_offset, void *grad_mask,
+                             dcn_stream_t stream) {
+    int Ho, Wo;
+    dcn_status s = check_core(p, &Ho, &Wo);
+    if (s != DCN_OK) return s;
+    if (p->B == 0) return DCN_OK;
+    if (!x || !offset || !mask || !grad_out || !grad_x || !grad_offset || !grad_mask)
+        return fail(DCN_ERR_NULL, "x, offset, mask, grad_out and the three gradients are required");
+    const size_t es = dtype_size(p->dtype);
+    if (!aligned(x, 16) || !aligned(grad_out, 16) || !aligned(grad_x, 16))
+        return fail(DCN_ERR_ALIGN, "x, grad_out and grad_x must be 16-byte aligned");
+    if (!aligned(offset, 2 * es) || !aligned(mask, es) || !aligned(grad_offset, 2 * es) || !aligned(grad_mask, es))
+        return fail(DCN_ERR_ALIGN, "offset/grad_offset need 2*sizeof(dtype), mask/grad_mask sizeof(dtype) alignment");
+    if (p->mask_mode == DCN_MASK_SOFTMAX && p->kh * p->kw > dcnb::kMaxSoftmaxK)
+        return fail(DCN_ERR_UNSUPPORTED, "softmax-mode backward supports K <= %d", dcnb::kMaxSoftmaxK);
+    dcnb::CoreArgs a = core_args(p, Ho, Wo);
+    a.x = x; a.offset = offset; a.mask = mask; a.grad_out = grad_out;
+    a.grad_x = grad_x; a.grad_offset = grad_offset; a.grad_mask = grad_mask;
+    return cuda_status(dcnb::launch_core_backward_generic(a, (cudaStream_t)stream), "dcn_core_backward launch");
+}
+
+dcn_status deform_agg_forward(const dagg_params *p, const void *feat, const int32_t *spatial_shape,
+                              const int32_t *scale_start_index, const float *sampling_location,
+                              const void *weights, void *out, dcn_stream_t stream) {
+    dcn_status s = check_agg(p);
+    if (s != DCN_OK) return s;
+    if (p->B == 0 || p->num_anchors == 0) return DCN_OK;
+    if (!feat || !spatial_shape || !scale_start_index || !sampling_location || !weights || !out)
+        return fail(DCN_ERR_NULL, "all tensor pointers are required");
+    const size_t es = dtype_size(p->dtype);
+    if (!aligned(feat, 16) || !aligned(out, 16)) return fail(DCN_ERR_ALIGN, "feat and out must be 16-byte aligned");
+    if (!aligned(sampling_location, 8) || !aligned(weights, es) || !aligned(spatial_shape, 4) ||
+        !aligned(scale_start_index, 4))
+        return fail(DCN_ERR_ALIGN, "sampling_location needs 8-byte, weights sizeof(dtype), tables 4-byte alignment");
+    dcnb::AggArgs a = agg_args(p);
+    a.feat = feat; a.spatial_shape = spatial_shape; a.scale_start = scale_start_index;
+    a.loc = sampling_location; a.weights = weights; a.out = out;
+    return cuda_status(dcnb::launch_agg_forward(a, (cudaStream_t)stream), "deform_agg_forward launch");
+}
+
+dcn_status deform_agg_backward(const dagg_params *p, const void *feat, const int32_t *spatial_shape,
+                               const int32_t *scale_start_index, const float *sampling_location,
+                               const void *weights, const void *grad_out, void *grad_feat, float *grad_loc,
+                               void *grad_weights, dcn_stream_t stream) {
+    dcn_status s = check_agg(p);
+    if (s != DCN_OK) return s;
+    if (p->B == 0 || p->num_anchors == 0) return DCN_OK;
+    if (!feat || !spatial_shape || !scale_start_index || !sampling_location || !weights || !grad_out ||
+        !grad_feat || !grad_loc || !grad_weights)
+        return fail(DCN_ERR_NULL, "all tensor pointers are required");
+    const size_t es = dtype_size(p->dtype);
+    if (!aligned(feat, 16) || !aligned(grad_out, 16) || !aligned(grad_feat, 16))
+        return fail(DCN_ERR_ALIGN, "feat, grad_out and grad_feat must be 16-byte aligned");
+    if (!aligned(sampling_location, 8) || !aligned(grad_loc, 8) || !aligned(weights, es) ||
+        !aligned(grad_weights, es) || !aligned(spatial_shape, 4) || !aligned(scale_start_index, 4))
+        return fail(DCN_ERR_ALIGN, "locations need 8-byte, weights sizeof(dtype), tables 4-byte alignment");
+    dcnb::AggArgs a = agg_args(p);
+    a.feat = feat; a.spatial_shape = spatial_shape; a.scale_start = scale_start_index;
+    a.loc = sampling_location; a.weights = weights; a.grad_out = grad_out;
+    a.grad_feat = grad_feat; a.grad_loc = grad_loc; a.grad_weights = grad_weights;
+    return cuda_status(dcnb::launch_agg_backward(a, (cudaStream_t)stream), "deform_agg_backward launch");
+}
+
+}  // extern "C"

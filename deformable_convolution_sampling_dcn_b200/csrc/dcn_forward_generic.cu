@@ -1,0 +1,140 @@
+// Generic forward core: any shape the ABI accepts.
+//
+// Work mapping: one sub-warp of LPI lanes per (pixel, group) item; lane s of
+// the sub-warp owns channels [s*V, (s+1)*V) of the group, V = 16 bytes of the
+// storage type, so every bilinear corner fetch is one 16-byte load per lane
+// and the LPI lanes of an item together read the C-contiguous corner row.
+// Items are enumerated in output memory order (b, ho, wo, g), so a warp's
+// stores cover consecutive 16-byte chunks.  Out-of-map corners are skipped;
+// sampling follows the bilinear definition of the DCNv1 page (section 2) and
+// the modulation of the DCNv2 page (section 1) and the YOLOv11 + DCNv4 page
+// (section 1.1: softmax over K for DCNv3, raw for DCNv4).
+#include "dcn_common.cuh"
+#include "dcn_launch.h"
+
+namespace dcnb {
+namespace {
+
+template <typename T, int LPI, bool SOFTMAX>
+__global__ void __launch_bounds__(256) core_forward_generic(CoreArgs a) {
+    constexpr int V = Storage<T>::kVec;
+    constexpr int IPW = 32 / LPI;
+    const int lane = threadIdx.x & 31;
+    const int sub = lane % LPI;
+    const int slot = lane / LPI;
+    const int K = a.kh * a.kw;
+    const int GC = a.G * a.C;
+    const long long n_items = (long long)a.B * a.Ho * a.Wo * a.G;
+    const long long warps_total = (long long)gridDim.x * (blockDim.x >> 5);
+    const T *__restrict__ x = static_cast<const T *>(a.x);
+    const T *__restrict__ off = static_cast<const T *>(a.offset);
+    const T *__restrict__ msk = static_cast<const T *>(a.mask);
+    T *__restrict__ out = static_cast<T *>(a.out);
+
+    for (long long item = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * IPW + slot;
+         item < n_items; item += warps_total * IPW) {
+        long long t = item;
+        const int g = (int)(t % a.G);
+        t /= a.G;
+        const int wo = (int)(t % a.Wo);
+        t /= a.Wo;
+        const int ho = (int)(t % a.Ho);
+        const int b = (int)(t / a.Ho);
+        const T *o_item = off + item * K * 2;
+        const T *m_item = msk + item * K;
+
+        float mx = 0.0f, inv_sum = 1.0f;
+        if (SOFTMAX) {
+            mx = -INFINITY;
+            for (int k = 0; k < K; ++k) mx = fmaxf(mx, load_scalar(m_item + k));
+            float s = 0.0f;
+            for (int k = 0; k < K; ++k) s += expf(load_scalar(m_item + k) - mx);
+            inv_sum = 1.0f / s;
+        }
+
+        float acc[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = 0.0f;
+        bool nan_pos = false;
+        const T *xb = x + (long long)b * a.H * a.W * GC + g * a.C + sub * V;
+
+        for (int i = 0; i < a.kh; ++i) {
+            const int by = ho * a.sh - a.ph + i * a.dh;
+            for (int j = 0; j < a.kw; ++j) {
+                const int k = i * a.kw + j;
+                const int bx = wo * a.sw - a.pw + j * a.dw;
+                const float2 d = load_pair(o_item + 2 * k);
+                float m = load_scalar(m_item + k);
+                if (SOFTMAX) m = expf(m - mx) * inv_sum;
+                const float px = fmaf(a.offset_scale, d.x, (float)bx);
+                const float py = fmaf(a.offset_scale, d.y, (float)by);
+                Tap tp;
+                const int st = make_tap(py, px, a.H, a.W, tp);
+                if (st < 0) nan_pos = true;
+                if (st <= 0) continue;
+                const float hy = 1.0f - tp.ly, hx = 1.0f - tp.lx;
+                const float w[4] = {hy * hx * m, hy * tp.lx * m, tp.ly * hx * m, tp.ly * tp.lx * m};
+                const bool vy[2] = {tp.y0 >= 0, tp.y0 + 1 < a.H};
+                const bool vx[2] = {tp.x0 >= 0, tp.x0 + 1 < a.W};
+#pragma unroll
+                for (int cy = 0; cy < 2; ++cy) {
+#pragma unroll
+                    for (int cx = 0; cx < 2; ++cx) {
+                        if (!(vy[cy] && vx[cx])) continue;
+                        const T *p = xb + ((long long)(tp.y0 + cy) * a.W + (tp.x0 + cx)) * GC;
+                        float f[V];
+                        unpack16<T>(ld_nc16(p), f);
+#pragma unroll
+                        for (int v = 0; v < V; ++v) acc[v] = fmaf(w[cy * 2 + cx], f[v], acc[v]);
+                    }
+                }
+            }
+        }
+        if (nan_pos) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] = __int_as_float(0x7fc00000);
+        }
+        T *o = out + (((long long)b * a.Ho + ho) * a.Wo + wo) * GC + g * a.C + sub * V;
+        *reinterpret_cast<uint4 *>(o) = pack16<T>(acc);
+    }
+}
+
+template <typename T, int LPI>
+cudaError_t launch_lpi(const CoreArgs &a, cudaStream_t stream) {
+    const long long n_items = (long long)a.B * a.Ho * a.Wo * a.G;
+    const int threads = 256;
+    const long long items_per_block = (threads / 32) * (32 / LPI);
+    long long blocks = (n_items + items_per_block - 1) / items_per_block;
+    if (blocks > 148LL * 64) blocks = 148LL * 64;  // grid-stride beyond this
+    if (a.softmax)
+        core_forward_generic<T, LPI, true><<<(unsigned)blocks, threads, 0, stream>>>(a);
+    else
+        core_forward_generic<T, LPI, false><<<(unsigned)blocks, threads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_t(const CoreArgs &a, cudaStream_t stream) {
+    const int lpi = a.C * (int)sizeof(T) / 16;
+    switch (lpi) {
+        case 1: return launch_lpi<T, 1>(a, stream);
+        case 2: return launch_lpi<T, 2>(a, stream);
+        case 4: return launch_lpi<T, 4>(a, stream);
+        case 8: return launch_lpi<T, 8>(a, stream);
+        case 16: return launch_lpi<T, 16>(a, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_core_forward_generic(const CoreArgs &a, cudaStream_t stream) {
+    switch (a.dtype) {
+        case DType::F32: return launch_t<float>(a, stream);
+        case DType::F16: return launch_t<__half>(a, stream);
+        case DType::BF16: return launch_t<__nv_bfloat16>(a, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace dcnb

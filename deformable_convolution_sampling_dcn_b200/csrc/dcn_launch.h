@@ -1,0 +1,55 @@
+// Internal launcher interface between the C-ABI layer (dcn_abi.cu) and the
+// kernels.  Arguments are validated by the ABI layer before any launcher runs.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dcnb {
+
+enum class DType : int { F32 = 0, F16 = 1, BF16 = 2 };
+
+// Largest K for which the softmax-mode backward keeps per-point gradients.
+constexpr int kMaxSoftmaxK = 49;
+
+struct CoreArgs {
+    const void *x;
+    const void *offset;
+    const void *mask;
+    void *out;              // forward output
+    const void *grad_out;   // backward only
+    void *grad_x;           // backward only
+    void *grad_offset;      // backward only
+    void *grad_mask;        // backward only
+    int B, H, W, G, C, kh, kw, sh, sw, ph, pw, dh, dw, Ho, Wo;
+    float offset_scale;
+    bool softmax;
+    DType dtype;
+};
+
+struct AggArgs {
+    const void *feat;
+    const int32_t *spatial_shape;
+    const int32_t *scale_start;
+    const float *loc;
+    const void *weights;
+    void *out;
+    const void *grad_out;   // backward only
+    void *grad_feat;        // backward only
+    float *grad_loc;        // backward only
+    void *grad_weights;     // backward only
+    int B, cams, scales, rows, A, P, G, C;
+    DType dtype;
+};
+
+// Each launcher enqueues its kernel(s) on `stream` and returns the
+// cudaGetLastError() of the launch.
+cudaError_t launch_core_forward_generic(const CoreArgs &a, cudaStream_t stream);
+cudaError_t launch_core_backward_generic(const CoreArgs &a, cudaStream_t stream);
+// Shared-memory path; sets *handled = false (and launches nothing) when the
+// problem does not fit it.
+cudaError_t launch_core_forward_plane(const CoreArgs &a, cudaStream_t stream, bool *handled);
+cudaError_t launch_agg_forward(const AggArgs &a, cudaStream_t stream);
+cudaError_t launch_agg_backward(const AggArgs &a, cudaStream_t stream);
+
+}  // namespace dcnb

@@ -1,0 +1,179 @@
+/*
+ * dcn_b200.h - C ABI of the B200 (sm_100a) deformable sampling-aggregation
+ * library.
+ *
+ * The operator.  For every output pixel p and channel group g, K kernel
+ * points are sampled at p0 + pk + dpk, where pk is the regular kernel grid
+ * and dpk a learned fractional offset ("用PyTorch实战DCNv1：从零构建可变形卷积与ROI池化模块",
+ * section 1: y(p0) = sum_n w(pn) x(p0 + pn + dpn)).  Each sample is a bilinear
+ * interpolation of the NHWC input (same page, section 2:
+ * x(p) = sum_q G(q,p) x(q), G(q,p) = g(qx,px) g(qy,py), g(a,b) = max(0, 1-|a-b|),
+ * grid points outside the map hold zero).  Each sample is weighted by a
+ * per-point modulation (DCNv2 page "DCNv2实战：在YOLOv5中替换普通卷积...", section 1:
+ * sum_n m(pn) w(pn) x(p + pn + dpn)), either normalised by a softmax over the K
+ * points of the (pixel, group) as in DCNv3 or used raw as in DCNv4 (YOLOv11 +
+ * DCNv4 article, section 1.1), and the K samples are summed in fp32.  The
+ * dense weight w(pn) of DCNv1/v2 is not part of this library: it is a plain
+ * convolution the caller runs before or after.
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers to dense, C-contiguous buffers
+ *     owned by the caller.  The library never allocates or frees memory.
+ *   - Calls are asynchronous on `stream` (0 = the legacy default stream)
+ *     and never synchronise.  A non-OK status means nothing was enqueued,
+ *     except DCN_ERR_CUDA after a failed launch.
+ *   - Every argument check runs on the host before any launch; a failed
+ *     check returns its status and touches no memory.
+ *   - x, offset, mask, out (and the gradients) share the storage dtype given
+ *     in the params; accumulation is fp32; results are rounded once,
+ *     nearest-even, to the storage dtype.
+ *   - Layouts (row-major, last index fastest):
+ *       x      [B, H, W, G*C]          channel = g*C + c
+ *       offset [B, Ho, Wo, G, K, 2]    last dim (dx, dy) in input pixels
+ *       mask   [B, Ho, Wo, G, K]       raw modulation, or logits (softmax mode)
+ *       out    [B, Ho, Wo, G*C]
+ *     with K = kh*kw, kernel point k = i*kw + j (i along H),
+ *     Ho = (H + 2*pad_h - (dil_h*(kh-1) + 1)) / stride_h + 1 (floor), and
+ *     likewise Wo.  Kernel point (i,j) of output (ho,wo) samples
+ *       y = ho*stride_h - pad_h + i*dil_h + offset_scale*dy,
+ *       x = wo*stride_w - pad_w + j*dil_w + offset_scale*dx,
+ *     formed in fp32 with one rounding (fused multiply-add).
+ *   - A sampling position that is not a number makes its whole (pixel,
+ *     group) output NaN; positions whose four grid neighbours all lie
+ *     outside the map (including infinite ones) contribute exactly zero.
+ *   - Supported group widths: C*sizeof(dtype) in {16, 32, 64, 128, 256}
+ *     bytes, i.e. C in {4,8,16,32,64} for fp32 and {8,16,32,64,128} for
+ *     fp16/bf16.  Other C return DCN_ERR_UNSUPPORTED.
+ *   - x, out, grad_out and grad_x must be 16-byte aligned; offset and its
+ *     gradient aligned to 2*sizeof(dtype); mask and its gradient to
+ *     sizeof(dtype).  Otherwise DCN_ERR_ALIGN.
+ *   - A problem with no output elements (B == 0) is a no-op returning DCN_OK;
+ *     its pointers may be NULL.
+ */
+#ifndef DCN_B200_H
+#define DCN_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *dcn_stream_t;
+
+typedef enum {
+    DCN_OK = 0,
+    DCN_ERR_NULL = 1,        /* a required pointer is NULL */
+    DCN_ERR_SHAPE = 2,       /* inconsistent or non-positive sizes, Ho or Wo < 1 */
+    DCN_ERR_UNSUPPORTED = 3, /* valid but not implemented (group width, dtype, mode) */
+    DCN_ERR_ALIGN = 4,       /* a pointer is not aligned as required */
+    DCN_ERR_CUDA = 5         /* the CUDA runtime reported an error at launch */
+} dcn_status;
+
+typedef enum { DCN_F32 = 0, DCN_F16 = 1, DCN_BF16 = 2 } dcn_dtype;
+
+typedef enum {
+    DCN_MASK_RAW = 0,    /* DCNv2/DCNv4: the mask is the modulation itself */
+    DCN_MASK_SOFTMAX = 1 /* DCNv3: the mask holds logits, normalised over K */
+} dcn_mask_mode;
+
+typedef struct {
+    int32_t B, H, W, G, C;   /* batch, input height/width, groups, channels per group */
+    int32_t kh, kw;          /* kernel height/width */
+    int32_t stride_h, stride_w;
+    int32_t pad_h, pad_w;
+    int32_t dil_h, dil_w;
+    float offset_scale;      /* multiplies every offset (1.0 = offsets in pixels) */
+    int32_t mask_mode;       /* dcn_mask_mode */
+    int32_t dtype;           /* dcn_dtype: storage type of every tensor */
+} dcn_params;
+
+/* Output spatial size for `p`.  Returns DCN_ERR_SHAPE (and leaves the
+ * outputs untouched) when the sizes are invalid or Ho/Wo would be < 1. */
+dcn_status dcn_core_output_hw(const dcn_params *p, int32_t *Ho, int32_t *Wo);
+
+/*
+ * Forward core: out = sum_k m_k * bilinear(x, p_k) per (pixel, group).
+ * Reads x, offset, mask; overwrites every element of out.
+ */
+dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offset,
+                            const void *mask, void *out, dcn_stream_t stream);
+
+/*
+ * Backward core: gradients of L = <grad_out, out> with respect to x, offset
+ * and mask.  The Sparse4D article (section 4.2) scatters the input gradient
+ * with atomic adds and accumulates the position gradients per thread before
+ * one write; this library does the same on the GPU.
+ *   grad_x      [B, H, W, G*C]        m_k * G(q, p_k) * grad_out, summed over taps
+ *   grad_offset [B, Ho, Wo, G, K, 2]  offset_scale * m_k * <grad_out, d x(p_k)/d p>
+ *   grad_mask   [B, Ho, Wo, G, K]     <grad_out, x(p_k)>, through the softmax
+ *                                     Jacobian m_k (g_k - sum_j m_j g_j) in
+ *                                     softmax mode
+ * All three are overwritten (grad_x is zeroed on `stream` first).  The
+ * derivative of g at a grid line is taken from the right.  The order of the
+ * atomic additions is not fixed, so grad_x may differ in the last bits from
+ * run to run.  Supported: every dtype and both mask modes.
+ */
+dcn_status dcn_core_backward(const dcn_params *p, const void *x, const void *offset,
+                             const void *mask, const void *grad_out, void *grad_x,
+                             void *grad_offset, void *grad_mask, dcn_stream_t stream);
+
+/*
+ * Multi-camera, multi-scale deformable aggregation (Sparse4D
+ * deformable_aggregation article, sections 1, 2.1 and 2.2).
+ *   feat              [B, num_rows, G*C]   features of every camera and scale,
+ *                     flattened: camera cam, scale s occupies rows
+ *                     scale_start_index[cam][s] + y*W_s + x
+ *   spatial_shape     [num_cams, num_scales, 2] int32 (H_s, W_s), device memory
+ *   scale_start_index [num_cams, num_scales]    int32, device memory
+ *   sampling_location [B, A, P, num_cams, 2]    fp32 (u, v), normalised to [0,1]
+ *                     per camera; sampled at (u*W_s - 0.5, v*H_s - 0.5), fp32
+ *   weights           [B, A, P, num_cams, num_scales, G], used as given
+ *   out               [B, A, G*C]
+ * out[b,a,g*C+c] = sum_{p,cam,s} weights[b,a,p,cam,s,g] * bilinear(map(cam,s), pos)[g*C+c].
+ * Rows outside [0, num_rows) are never read: a table entry that points
+ * there contributes zero.  feat, weights and out share `dtype`; locations
+ * are always fp32.  Same group widths and alignment rules as the core.
+ */
+typedef struct {
+    int32_t B, num_cams, num_scales, num_rows, num_anchors, num_pts, G, C;
+    int32_t dtype; /* dcn_dtype */
+} dagg_params;
+
+dcn_status deform_agg_forward(const dagg_params *p, const void *feat,
+                              const int32_t *spatial_shape, const int32_t *scale_start_index,
+                              const float *sampling_location, const void *weights, void *out,
+                              dcn_stream_t stream);
+
+/*
+ * Aggregation backward: gradients of <grad_out, out>.
+ *   grad_feat    [B, num_rows, G*C]     scatter of weight * G(q,p) * grad_out (atomic)
+ *   grad_loc     [B, A, P, num_cams, 2] fp32; sum over scales and groups of
+ *                weight * W_s (resp. H_s) * <grad_out, d x / d px (resp. py)>
+ *   grad_weights [B, A, P, num_cams, num_scales, G]  <grad_out, sample>
+ * All three are overwritten (grad_feat is zeroed on `stream` first).
+ */
+dcn_status deform_agg_backward(const dagg_params *p, const void *feat,
+                               const int32_t *spatial_shape, const int32_t *scale_start_index,
+                               const float *sampling_location, const void *weights,
+                               const void *grad_out, void *grad_feat, float *grad_loc,
+                               void *grad_weights, dcn_stream_t stream);
+
+/* Static, human-readable name of a status. */
+const char *dcn_status_string(dcn_status s);
+
+/* Detail of the last non-OK status returned on the calling thread (which
+ * check failed, or the CUDA error string).  Never NULL. */
+const char *dcn_last_error_detail(void);
+
+/* ABI version of this header (bumped on any incompatible change). */
+int32_t dcn_abi_version(void);
+
+#define DCN_ABI_VERSION 1
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCN_B200_H */
