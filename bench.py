@@ -139,6 +139,16 @@ def build_sets(shape, seed, dev, l2_bytes):
     return inp, sets, R, footprint
 
 
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The largest `value` over all ranks (the job is as slow as its slowest
+    rank); identity on one process."""
+    if world <= 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 def capture(fn_list, stream):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
@@ -174,11 +184,7 @@ def time_steps(make_call, sets, K, W, stream, barrier, world):
         e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
     del g_full, g_rem
     return ms
 
@@ -300,11 +306,7 @@ def measure_e2e(dcn, shape, inp, dev, stream, E, barrier, world):
         e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
     h2d = sum(t.numel() * t.element_size() for t in (hx, hoff, hm))
     d2h = hout.numel() * hout.element_size()
     return {"value": round(shape.samples * world / (ms / 1e3 / E) / 1e9, 3), "unit": "Gsamples/s",

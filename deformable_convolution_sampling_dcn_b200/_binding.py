@@ -25,7 +25,8 @@ _DTYPE_CODE = {torch.float32: DCN_F32, torch.float16: DCN_F16, torch.bfloat16: D
 
 # Every entry point include/dcn_b200.h declares.
 EXPORTS = ("dcn_core_output_hw", "dcn_core_forward", "dcn_core_backward", "deform_agg_forward",
-           "deform_agg_backward", "dcn_status_string", "dcn_last_error_detail", "dcn_abi_version")
+           "deform_agg_backward", "dcn_status_string", "dcn_last_error_detail", "dcn_abi_version",
+           "dcn_take_device_error")
 ABI_VERSION = 1
 
 
@@ -69,6 +70,8 @@ def _declare(lib):
     lib.dcn_last_error_detail.restype = ctypes.c_char_p
     lib.dcn_abi_version.argtypes = []
     lib.dcn_abi_version.restype = ctypes.c_int32
+    lib.dcn_take_device_error.argtypes = []
+    lib.dcn_take_device_error.restype = ctypes.c_int32
     return lib
 
 
@@ -130,6 +133,11 @@ def core_params(x: torch.Tensor, G: int, kernel=(3, 3), stride=(1, 1), pad=(1, 1
     dh, dw = _pair(dil)
     return DcnParams(B, H, W, G, GC // G, kh, kw, sh, sw, ph, pw, dh, dw, float(offset_scale),
                      DCN_MASK_SOFTMAX if softmax else DCN_MASK_RAW, _DTYPE_CODE[x.dtype])
+
+
+def take_device_error() -> int:
+    """Read and clear the device error word (0 = no bounded wait ran out)."""
+    return int(lib().dcn_take_device_error())
 
 
 def dcn_core_output_hw(p: DcnParams) -> Tuple[int, int]:

@@ -4,6 +4,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "../../include/dcn_b200.h"
@@ -104,6 +105,12 @@ extern "C" {
 
 int32_t dcn_abi_version(void) { return DCN_ABI_VERSION; }
 
+int32_t dcn_take_device_error(void) {
+    unsigned int v = 0;
+    if (dcnb::take_device_error(&v) != cudaSuccess) return -1;
+    return (int32_t)v;
+}
+
 const char *dcn_last_error_detail(void) { return g_detail; }
 
 const char *dcn_status_string(dcn_status s) {
@@ -142,7 +149,9 @@ dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offs
     dcnb::CoreArgs a = core_args(p, Ho, Wo);
     a.x = x; a.offset = offset; a.mask = mask; a.out = out;
     bool handled = false;
-    cudaError_t e = dcnb::launch_core_forward_plane(a, (cudaStream_t)stream, &handled);
+    cudaError_t e = cudaSuccess;
+    const char *force = getenv("DCN_B200_FORCE_GENERIC");
+    if (!(force && force[0] == '1')) e = dcnb::launch_core_forward_plane(a, (cudaStream_t)stream, &handled);
     if (!handled) e = dcnb::launch_core_forward_generic(a, (cudaStream_t)stream);
     return cuda_status(e, "dcn_core_forward launch");
 }

@@ -49,6 +49,9 @@ cudaError_t launch_core_backward_generic(const CoreArgs &a, cudaStream_t stream)
 // Shared-memory path; sets *handled = false (and launches nothing) when the
 // problem does not fit it.
 cudaError_t launch_core_forward_plane(const CoreArgs &a, cudaStream_t stream, bool *handled);
+// Reads and clears the device error word that bounded waits set (bit 0:
+// a TMA wait ran out).  Synchronous.
+cudaError_t take_device_error(unsigned int *value);
 cudaError_t launch_agg_forward(const AggArgs &a, cudaStream_t stream);
 cudaError_t launch_agg_backward(const AggArgs &a, cudaStream_t stream);
 

@@ -96,6 +96,11 @@ dcn_status dcn_core_output_hw(const dcn_params *p, int32_t *Ho, int32_t *Wo);
 /*
  * Forward core: out = sum_k m_k * bilinear(x, p_k) per (pixel, group).
  * Reads x, offset, mask; overwrites every element of out.
+ * Two kernels implement it: a shared-memory staged one (group rows of 32 to
+ * 256 bytes, W <= 254, K <= 64) and a generic one for every other shape.
+ * Setting the environment variable DCN_B200_FORCE_GENERIC=1 routes every
+ * call to the generic kernel (both give the same result up to fp32
+ * summation order).
  */
 dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offset,
                             const void *mask, void *out, dcn_stream_t stream);
@@ -166,6 +171,13 @@ const char *dcn_status_string(dcn_status s);
 /* Detail of the last non-OK status returned on the calling thread (which
  * check failed, or the CUDA error string).  Never NULL. */
 const char *dcn_last_error_detail(void);
+
+/* Device-side error word: kernels that wait on their own asynchronous
+ * copies bound every wait (1 s); if one ran out the kernel sets bit 0 of this
+ * word and returns without finishing its outputs.  This call synchronises
+ * the device, returns the word and clears it; -1 if the read itself failed.
+ * 0 after every normal run. */
+int32_t dcn_take_device_error(void);
 
 /* ABI version of this header (bumped on any incompatible change). */
 int32_t dcn_abi_version(void);

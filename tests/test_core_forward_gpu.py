@@ -80,6 +80,43 @@ def test_small_ragged(case, cuda_dev):
     assert_close_fwd(out, ref, f"small case {case}")
 
 
+@pytest.mark.parametrize("name", ["dcnv3_tiny", "dcnv4_p4", "dcnv3_p3_dil2"])
+def test_generic_path_full_size(name, cuda_dev, monkeypatch):
+    """The generic kernel on the shapes the staged kernel normally takes."""
+    monkeypatch.setenv("DCN_B200_FORCE_GENERIC", "1")
+    shape, inp = si.workload_core(name)
+    out, ref = run_case(shape, inp, cuda_dev)
+    assert_close_fwd(out, ref, name + " generic")
+
+
+@pytest.mark.parametrize("dt", ["f32", "f16", "bf16"])
+def test_far_offsets_many_segments(dt, cuda_dev):
+    """Offsets far beyond the staged halo (std 12 px) on a tall map: many taps
+    take the direct global-memory path and every CTA walks several segments."""
+    shape = si.CoreShape(B=2, H=150, W=37, G=2, C=32, dtype=dt, softmax=(dt == "bf16"))
+    inp = si.core_inputs(shape, 11, offset_std=12.0, oob_fraction=0.02)
+    out, ref = run_case(shape, inp, cuda_dev)
+    assert_close_fwd(out, ref, "far offsets")
+    d = dcn()
+    assert d._binding.take_device_error() == 0
+
+
+def test_strided_dilated_staged(cuda_dev):
+    shape = si.CoreShape(B=3, H=61, W=45, G=3, C=16, kh=5, kw=3, stride_h=2, stride_w=3, pad_h=4, pad_w=2,
+                         dil_h=2, dil_w=2, offset_scale=0.4, softmax=True, dtype="f16")
+    inp = si.core_inputs(shape, 12, offset_std=3.0)
+    out, ref = run_case(shape, inp, cuda_dev)
+    assert_close_fwd(out, ref, "strided dilated")
+
+
+def test_wide_pad_no_rows_staged(cuda_dev):
+    """Padding so wide that some segments stage no input rows at all."""
+    shape = si.CoreShape(B=1, H=9, W=11, G=2, C=32, kh=3, kw=3, pad_h=15, pad_w=3, dtype="f32")
+    inp = si.core_inputs(shape, 13, offset_std=2.0)
+    out, ref = run_case(shape, inp, cuda_dev)
+    assert_close_fwd(out, ref, "wide pad")
+
+
 def test_large_map(cuda_dev):
     """A 1024 x 1024 map (narrow groups): many tiles and a long grid-stride loop."""
     shape = si.CoreShape(B=1, H=1024, W=1024, G=1, C=8, dtype="f16")
