@@ -7,7 +7,7 @@
 #include <stdlib.h>
 #include <string.h>
 
-#include "../../include/dcn_b200.h"
+#include "dcn_b200.h"
 #include "dcn_launch.h"
 
 namespace {

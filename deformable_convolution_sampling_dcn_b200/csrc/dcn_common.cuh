@@ -70,6 +70,26 @@ template <> __device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4 
     }
 }
 
+// Unpack a 16-byte vector into V/2 fp32 pairs (for packed fp32x2 math).
+template <typename T> __device__ __forceinline__ void unpack16x2(const uint4 &v, float2 *f);
+template <> __device__ __forceinline__ void unpack16x2<float>(const uint4 &v, float2 *f) {
+    f[0] = make_float2(__uint_as_float(v.x), __uint_as_float(v.y));
+    f[1] = make_float2(__uint_as_float(v.z), __uint_as_float(v.w));
+}
+template <> __device__ __forceinline__ void unpack16x2<__half>(const uint4 &v, float2 *f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        asm("{.reg .f16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;}"
+            : "=f"(f[i].x), "=f"(f[i].y)
+            : "r"(w[i]));
+}
+template <> __device__ __forceinline__ void unpack16x2<__nv_bfloat16>(const uint4 &v, float2 *f) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+}
+
 // Pack fp32 values into a 16-byte vector, rounding nearest-even.
 template <typename T> __device__ __forceinline__ uint4 pack16(const float *f);
 template <> __device__ __forceinline__ uint4 pack16<float>(const float *f) {
