@@ -53,6 +53,9 @@ cudaError_t launch_core_forward_plane(const CoreArgs &a, cudaStream_t stream, bo
 // a TMA wait ran out).  Synchronous.
 cudaError_t take_device_error(unsigned int *value);
 cudaError_t launch_agg_forward(const AggArgs &a, cudaStream_t stream);
+// Anchor-wide aggregation kernels (all groups per CTA); sets *handled = false
+// (and launches nothing) when the feature row width does not fit them.
+cudaError_t launch_agg_wide(const AggArgs &a, bool bwd, cudaStream_t stream, bool *handled);
 cudaError_t launch_agg_backward(const AggArgs &a, cudaStream_t stream);
 
 }  // namespace dcnb

@@ -8,6 +8,8 @@
 // bilinear corner fetch is one 16-byte load per lane over a C-contiguous row
 // of the flattened [B, rows, G*C] features.  Partial sums of the sub-warps
 // are combined with shuffles at the end (forward) or per pair (backward).
+#include <stdlib.h>
+
 #include "dcn_atomic.cuh"
 #include "dcn_launch.h"
 
@@ -230,7 +232,24 @@ cudaError_t dispatch_dtype(const AggArgs &a, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_agg_forward(const AggArgs &a, cudaStream_t stream) { return dispatch_dtype<false>(a, stream); }
-cudaError_t launch_agg_backward(const AggArgs &a, cudaStream_t stream) { return dispatch_dtype<true>(a, stream); }
+cudaError_t launch_agg_forward(const AggArgs &a, cudaStream_t stream) {
+    bool handled = false;
+    const char *force = getenv("DCN_B200_FORCE_GENERIC");
+    if (!(force && force[0] == '1')) {
+        const cudaError_t e = launch_agg_wide(a, false, stream, &handled);
+        if (handled) return e;
+    }
+    return dispatch_dtype<false>(a, stream);
+}
+
+cudaError_t launch_agg_backward(const AggArgs &a, cudaStream_t stream) {
+    bool handled = false;
+    const char *force = getenv("DCN_B200_FORCE_GENERIC");
+    if (!(force && force[0] == '1')) {
+        const cudaError_t e = launch_agg_wide(a, true, stream, &handled);
+        if (handled) return e;
+    }
+    return dispatch_dtype<true>(a, stream);
+}
 
 }  // namespace dcnb

@@ -1,0 +1,273 @@
+// Multi-camera multi-scale aggregation, anchor-wide kernels (Sparse4D
+// deformable_aggregation article, sections 1, 2.1, 2.2 and 4).
+//
+// The sampling position of (anchor, point, camera, scale) does not depend on
+// the group, so one CTA handles one (b, anchor) with all G groups at once:
+// the tap geometry (corner rows, bilinear weights) is computed once per
+// sample instead of once per group, and each bilinear corner of all groups is
+// one contiguous G*C row that the 32 lanes of a warp read as CPL coalesced
+// 512-byte transactions (lane l, chunk j owns elements (32*j + l)*V ...).
+// The CTA's warps split the anchor's (point, camera) pairs; each warp walks
+// the scales of its pairs, and the warps' partial rows are summed through
+// shared memory at the end (forward).  In the backward each pair belongs to
+// exactly one warp, so the location gradient of a pair is reduced inside the
+// warp and stored without atomics; the weight gradient of (sample, group) is
+// reduced over the lanes of the group; the feature gradient is scattered with
+// 16-byte vector reductions.
+//
+// Taken when G*C*sizeof(T) is 512, 1024 or 2048 bytes; other widths use the
+// per-group kernels in deform_agg.cu.
+#include "dcn_atomic.cuh"
+#include "dcn_launch.h"
+
+namespace dcnb {
+namespace {
+
+constexpr int kAggWarps = 8;        // warps per anchor CTA
+constexpr int kAggTableMax = 512;   // (camera, scale) entries cached in shared memory
+
+__device__ __forceinline__ int4 load_table(const AggArgs &a, int cs) {
+    return make_int4(__ldg(a.spatial_shape + 2 * cs), __ldg(a.spatial_shape + 2 * cs + 1), __ldg(a.scale_start + cs), 0);
+}
+
+template <typename T, int CPL>
+__global__ void __launch_bounds__(kAggWarps * 32) agg_forward_wide(AggArgs a) {
+    constexpr int V = Storage<T>::kVec;
+    constexpr int ROW = CPL * 32 * V;  // elements in one feature row (G*C)
+    __shared__ int4 tab[kAggTableMax];
+    __shared__ float part[kAggWarps][ROW];
+    __shared__ int nan_any;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int CS = a.cams * a.scales;
+    const bool tab_smem = CS <= kAggTableMax;
+    if (tab_smem)
+        for (int i = threadIdx.x; i < CS; i += blockDim.x) tab[i] = load_table(a, i);
+    if (threadIdx.x == 0) nan_any = 0;
+    __syncthreads();
+
+    const long long ba = blockIdx.x;  // b * A + anchor
+    const int b = (int)(ba / a.A);
+    const T *__restrict__ feat = static_cast<const T *>(a.feat) + (long long)b * a.rows * ROW;
+    const T *__restrict__ wts = static_cast<const T *>(a.weights);
+    const int pairs = a.P * a.cams;
+    int grp[CPL];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) grp[j] = (32 * j + lane) * V / a.C;
+    float acc[CPL][V];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j)
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[j][v] = 0.0f;
+    bool nan_pos = false;
+
+    for (int pc = warp; pc < pairs; pc += kAggWarps) {
+        const int cam = pc % a.cams;
+        const float2 uv = __ldg(reinterpret_cast<const float2 *>(a.loc) + ba * pairs + pc);
+        const long long wbase = (ba * pairs + pc) * a.scales;
+#pragma unroll 4
+        for (int s = 0; s < a.scales; ++s) {
+            const int4 t = tab_smem ? tab[cam * a.scales + s] : load_table(a, cam * a.scales + s);
+            const float px = fmaf(uv.x, (float)t.y, -0.5f);
+            const float py = fmaf(uv.y, (float)t.x, -0.5f);
+            Tap tp{0, 0, 0.0f, 0.0f};
+            const int st = make_tap(py, px, t.x, t.y, tp);
+            if (st < 0) nan_pos = true;
+            if (st <= 0) continue;
+            float w[CPL];
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) w[j] = load_scalar(wts + (wbase + s) * a.G + grp[j]);
+            const float gyv[2] = {1.0f - tp.ly, tp.ly};
+            const float gxv[2] = {1.0f - tp.lx, tp.lx};
+#pragma unroll
+            for (int cy = 0; cy < 2; ++cy) {
+#pragma unroll
+                for (int cx = 0; cx < 2; ++cx) {
+                    const int y = tp.y0 + cy, x = tp.x0 + cx;
+                    if (y < 0 || y >= t.x || x < 0 || x >= t.y) continue;
+                    const long long row = (long long)t.z + (long long)y * t.y + x;
+                    if (row < 0 || row >= a.rows) continue;
+                    const float g = gyv[cy] * gxv[cx];
+                    const T *r = feat + row * ROW + lane * V;
+#pragma unroll
+                    for (int j = 0; j < CPL; ++j) {
+                        float f[V];
+                        unpack16<T>(ld_nc16(r + 32 * j * V), f);
+                        const float wg = w[j] * g;
+#pragma unroll
+                        for (int v = 0; v < V; ++v) acc[j][v] = fmaf(wg, f[v], acc[j][v]);
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < CPL; ++j)
+#pragma unroll
+        for (int v = 0; v < V; ++v) part[warp][(32 * j + lane) * V + v] = acc[j][v];
+    if (nan_pos) atomicOr(&nan_any, 1);
+    __syncthreads();
+    // sum the warps' partial rows; each thread produces 16-byte chunks
+    T *__restrict__ out = static_cast<T *>(a.out) + ba * ROW;
+    for (int c = threadIdx.x; c < ROW / V; c += blockDim.x) {
+        float f[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) {
+            float sum = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kAggWarps; ++w) sum += part[w][c * V + v];
+            f[v] = nan_any ? __int_as_float(0x7fc00000) : sum;
+        }
+        *reinterpret_cast<uint4 *>(out + c * V) = pack16<T>(f);
+    }
+}
+
+template <typename T, int CPL>
+__global__ void __launch_bounds__(kAggWarps * 32) agg_backward_wide(AggArgs a) {
+    constexpr int V = Storage<T>::kVec;
+    constexpr int ROW = CPL * 32 * V;
+    __shared__ int4 tab[kAggTableMax];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int CS = a.cams * a.scales;
+    const bool tab_smem = CS <= kAggTableMax;
+    if (tab_smem)
+        for (int i = threadIdx.x; i < CS; i += blockDim.x) tab[i] = load_table(a, i);
+    __syncthreads();
+
+    const long long ba = blockIdx.x;
+    const int b = (int)(ba / a.A);
+    const long long fofs = (long long)b * a.rows * ROW;
+    const T *__restrict__ feat = static_cast<const T *>(a.feat) + fofs;
+    T *__restrict__ gfeat = static_cast<T *>(a.grad_feat) + fofs;
+    const T *__restrict__ wts = static_cast<const T *>(a.weights);
+    T *__restrict__ gw = static_cast<T *>(a.grad_weights);
+    const int pairs = a.P * a.cams;
+    // lanes of one group inside a chunk: C / V consecutive lanes (aligned)
+    const int gl = a.C / V;  // 1..32, a power of two
+    int grp[CPL];
+    float go[CPL][V];
+    const T *gout = static_cast<const T *>(a.grad_out) + ba * ROW;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        grp[j] = (32 * j + lane) * V / a.C;
+        unpack16<T>(ld_nc16(gout + (32 * j + lane) * V), go[j]);
+    }
+
+    for (int pc = warp; pc < pairs; pc += kAggWarps) {
+        const int cam = pc % a.cams;
+        const float2 uv = __ldg(reinterpret_cast<const float2 *>(a.loc) + ba * pairs + pc);
+        const long long wbase = (ba * pairs + pc) * a.scales;
+        float glx = 0.0f, gly = 0.0f;
+        bool nan_pos = false;
+        for (int s = 0; s < a.scales; ++s) {
+            const int4 t = tab_smem ? tab[cam * a.scales + s] : load_table(a, cam * a.scales + s);
+            const float px = fmaf(uv.x, (float)t.y, -0.5f);
+            const float py = fmaf(uv.y, (float)t.x, -0.5f);
+            Tap tp{0, 0, 0.0f, 0.0f};
+            const int st = make_tap(py, px, t.x, t.y, tp);
+            float w[CPL];
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) w[j] = load_scalar(wts + (wbase + s) * a.G + grp[j]);
+            float val[CPL], dpx[CPL], dpy[CPL];
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) val[j] = dpx[j] = dpy[j] = 0.0f;
+            if (st > 0) {
+                const float gyv[2] = {1.0f - tp.ly, tp.ly};
+                const float gxv[2] = {1.0f - tp.lx, tp.lx};
+#pragma unroll
+                for (int cy = 0; cy < 2; ++cy) {
+#pragma unroll
+                    for (int cx = 0; cx < 2; ++cx) {
+                        const int y = tp.y0 + cy, x = tp.x0 + cx;
+                        if (y < 0 || y >= t.x || x < 0 || x >= t.y) continue;
+                        const long long row = (long long)t.z + (long long)y * t.y + x;
+                        if (row < 0 || row >= a.rows) continue;
+                        const float G = gyv[cy] * gxv[cx];
+                        const float sx = cx ? gyv[cy] : -gyv[cy];
+                        const float sy = cy ? gxv[cx] : -gxv[cx];
+#pragma unroll
+                        for (int j = 0; j < CPL; ++j) {
+                            const long long e = row * ROW + (32 * j + lane) * V;
+                            float f[V];
+                            unpack16<T>(ld_nc16(feat + e), f);
+                            float dc = 0.0f;
+#pragma unroll
+                            for (int v = 0; v < V; ++v) dc = fmaf(go[j][v], f[v], dc);
+                            val[j] = fmaf(G, dc, val[j]);
+                            dpx[j] = fmaf(sx, dc, dpx[j]);
+                            dpy[j] = fmaf(sy, dc, dpy[j]);
+                            const float wg = w[j] * G;
+                            float c[V];
+#pragma unroll
+                            for (int v = 0; v < V; ++v) c[v] = wg * go[j][v];
+                            red_add16<T>(gfeat + e, c);
+                        }
+                    }
+                }
+            }
+            if (st < 0) nan_pos = true;
+            // weight gradient of (sample, group): sum over the group's lanes
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                float v = val[j];
+                for (int o = 1; o < gl; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (st < 0) v = __int_as_float(0x7fc00000);
+                if ((lane & (gl - 1)) == 0) gw[(wbase + s) * a.G + grp[j]] = from_f32<T>(v);
+                glx = fmaf(w[j] * (float)t.y, dpx[j], glx);
+                gly = fmaf(w[j] * (float)t.x, dpy[j], gly);
+            }
+        }
+        // location gradient of the pair: all groups and scales, one warp
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            glx += __shfl_xor_sync(0xffffffffu, glx, o);
+            gly += __shfl_xor_sync(0xffffffffu, gly, o);
+        }
+        nan_pos = __any_sync(0xffffffffu, nan_pos);
+        if (lane == 0) {
+            const float nan = __int_as_float(0x7fc00000);
+            reinterpret_cast<float2 *>(a.grad_loc)[ba * pairs + pc] =
+                nan_pos ? make_float2(nan, nan) : make_float2(glx, gly);
+        }
+    }
+}
+
+template <typename T, int CPL>
+cudaError_t launch(const AggArgs &a, bool bwd, cudaStream_t stream) {
+    const unsigned grid = (unsigned)((long long)a.B * a.A);
+    if (bwd) {
+        cudaError_t e = cudaMemsetAsync(a.grad_feat, 0, (size_t)a.B * a.rows * a.G * a.C * sizeof(T), stream);
+        if (e != cudaSuccess) return e;
+        agg_backward_wide<T, CPL><<<grid, kAggWarps * 32, 0, stream>>>(a);
+    } else {
+        agg_forward_wide<T, CPL><<<grid, kAggWarps * 32, 0, stream>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_t(const AggArgs &a, bool bwd, cudaStream_t stream, bool *handled) {
+    const long long row_bytes = (long long)a.G * a.C * sizeof(T);
+    if ((long long)a.B * a.A > 0x7fffffffLL) return cudaSuccess;
+    *handled = true;
+    switch (row_bytes) {
+        case 512: return launch<T, 1>(a, bwd, stream);
+        case 1024: return launch<T, 2>(a, bwd, stream);
+        case 2048: return launch<T, 4>(a, bwd, stream);
+    }
+    *handled = false;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_agg_wide(const AggArgs &a, bool bwd, cudaStream_t stream, bool *handled) {
+    *handled = false;
+    switch (a.dtype) {
+        case DType::F32: return launch_t<float>(a, bwd, stream, handled);
+        case DType::F16: return launch_t<__half>(a, bwd, stream, handled);
+        case DType::BF16: return launch_t<__nv_bfloat16>(a, bwd, stream, handled);
+    }
+    return cudaSuccess;
+}
+
+}  // namespace dcnb

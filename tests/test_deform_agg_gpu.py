@@ -20,6 +20,24 @@ def run_fwd(inp, dev):
     return out, ref
 
 
+def test_sparse4d_full_size_generic(cuda_dev, monkeypatch):
+    """The per-group kernels on the shape the anchor-wide kernels normally take."""
+    monkeypatch.setenv("DCN_B200_FORCE_GENERIC", "1")
+    inp = si.agg_inputs(si.SPARSE4D, si.SEEDS["sparse4d"])
+    out, ref = run_fwd(inp, cuda_dev)
+    assert_close_fwd(out, ref, "sparse4d generic")
+
+
+def test_sparse4d_backward_generic(cuda_dev, monkeypatch):
+    monkeypatch.setenv("DCN_B200_FORCE_GENERIC", "1")
+    shape = si.AggShape(B=1, num_cams=3, scales=((16, 44), (8, 22)), num_anchors=40, num_pts=5, G=8, C=32)
+    inp = si.agg_inputs(shape, 77, with_grad_out=True, loc_lo=-0.05, loc_hi=1.05)
+    (gf, gl, gw), ref = run_bwd(inp, cuda_dev)
+    assert_close_bwd(gf, ref["grad_feat"], "grad_feat")
+    assert_close_bwd(gw, ref["grad_weights"], "grad_weights")
+    assert_close_bwd(gl, ref["grad_loc"], "grad_loc")
+
+
 def test_sparse4d_full_size(cuda_dev):
     inp = si.agg_inputs(si.SPARSE4D, si.SEEDS["sparse4d"])
     out, ref = run_fwd(inp, cuda_dev)
@@ -30,6 +48,9 @@ def test_sparse4d_full_size(cuda_dev):
 SMALL = [
     # B, cams, scales, A, P, G, C, dtype, loc range
     (1, 2, ((5, 7), (3, 4)), 3, 2, 2, 8, "f32", (-0.1, 1.1)),
+    (2, 3, ((7, 9), (3, 5)), 11, 3, 4, 32, "f32", (-0.1, 1.1)),      # 512-byte rows: anchor-wide
+    (1, 2, ((6, 10),), 9, 4, 8, 64, "f16", (-0.1, 1.1)),             # 1024-byte rows: anchor-wide
+    (1, 4, ((5, 6), (4, 3), (2, 2)), 7, 2, 16, 64, "bf16", (0.0, 1.0)),  # 2048-byte rows
     (2, 3, ((9, 13), (4, 6), (2, 3)), 17, 5, 4, 32, "f32", (0.0, 1.0)),
     (1, 6, ((16, 44), (8, 22)), 50, 13, 8, 32, "f16", (-0.05, 1.05)),
     (2, 1, ((10, 10),), 9, 3, 1, 64, "bf16", (-0.2, 1.2)),
