@@ -67,6 +67,8 @@ def _bind(lib):
     lib.oracle_agg_forward.restype = None
     lib.oracle_agg_backward.argtypes = [i] * 8 + [dp, ip, ip, fp, dp, dp, dp, dp, dp]
     lib.oracle_agg_backward.restype = None
+    lib.oracle_roi_pool_forward.argtypes = [i] * 8 + [ctypes.c_float, ctypes.c_float, dp, fp, fp, dp]
+    lib.oracle_roi_pool_forward.restype = None
     return lib
 
 
@@ -177,3 +179,26 @@ def agg_backward(feat, spatial_shape, scale_start_index, sampling_location, weig
                             _ptr(go, ctypes.c_double), _ptr(gf, ctypes.c_double),
                             _ptr(gl, ctypes.c_double), _ptr(gw, ctypes.c_double))
     return {"grad_feat": gf, "grad_loc": gl, "grad_weights": gw}
+
+
+def roi_pool_forward(x, rois, offset, *, pooled=(7, 7), sampling=2, spatial_scale: float = 1.0,
+                     gamma: float = 0.1, lib=None) -> np.ndarray:
+    """out [N, PH, PW, C] (fp64) of deformable RoI pooling over x [B, H, W, C].
+
+    rois [N, 5] (batch, x1, y1, x2, y2) and offset [N, PH, PW, 2] are fp32."""
+    lib = lib or load()
+    x = _f64(x)
+    B, H, W, C = x.shape
+    r = rois.detach().cpu().numpy() if hasattr(rois, "detach") else rois
+    o = offset.detach().cpu().numpy() if hasattr(offset, "detach") else offset
+    r = np.ascontiguousarray(r, dtype=np.float32)
+    o = np.ascontiguousarray(o, dtype=np.float32)
+    N = r.shape[0]
+    PH, PW = pooled
+    assert r.shape == (N, 5) and o.shape == (N, PH, PW, 2)
+    assert np.all((r[:, 0] >= 0) & (r[:, 0] < B) & (r[:, 0] == np.floor(r[:, 0])))
+    out = np.empty((N, PH, PW, C), dtype=np.float64)
+    lib.oracle_roi_pool_forward(B, H, W, C, N, PH, PW, int(sampling), float(spatial_scale), float(gamma),
+                                _ptr(x, ctypes.c_double), _ptr(r, ctypes.c_float), _ptr(o, ctypes.c_float),
+                                _ptr(out, ctypes.c_double))
+    return out

@@ -365,3 +365,68 @@ void oracle_agg_backward(int B, int cams, int S, int rows, int A, int P, int G, 
         for (size_t i = 0; i < nl; ++i) grad_loc[i] += gl_part[(size_t)g * nl + i];
     free(gl_part);
 }
+
+/*
+ * Deformable RoI pooling, forward ("用PyTorch实战DCNv1：从零构建可变形卷积与ROI池化模块",
+ * section 3): the k x k bins of a region of interest are each moved by a
+ * learned offset normalised by the region size, dp = gamma * dp_hat o (w, h),
+ * and each bin's value is read by bilinear interpolation (the same kernel
+ * g(a,b) = max(0, 1-|a-b|) as the core, zeros outside the map).
+ *   x      [B, H, W, C]
+ *   rois   [N, 5]      (batch index, x1, y1, x2, y2) in input-image units
+ *   offset [N, PH, PW, 2]  (dx_hat, dy_hat), normalised by the region size
+ *   out    [N, PH, PW, C]
+ * Reading (the page gives the offset normalisation and the interpolation
+ * only): coordinates are scaled by spatial_scale, the region is at least one
+ * pixel on each side, each bin averages S x S sampling points placed at the
+ * centres of an S x S sub-grid of the bin, pixel centres at integers.  All
+ * position arithmetic is fp32 with one rounding per operation, in this
+ * order, so that both implementations take the same floor() decisions.
+ */
+void oracle_roi_pool_forward(int B, int H, int W, int C, int N, int PH, int PW, int S,
+                             float spatial_scale, float gamma,
+                             const double *x, const float *rois, const float *offset, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        const float *r = rois + (size_t)n * 5;
+        const int b = (int)r[0];
+        const float x1 = r[1] * spatial_scale, y1 = r[2] * spatial_scale;
+        const float x2 = r[3] * spatial_scale, y2 = r[4] * spatial_scale;
+        float rw = x2 - x1, rh = y2 - y1;
+        if (!(rw >= 1.0f)) rw = 1.0f;
+        if (!(rh >= 1.0f)) rh = 1.0f;
+        const float bw = rw / (float)PW, bh = rh / (float)PH;
+        const float sw = bw / (float)S, sh = bh / (float)S;
+        for (int i = 0; i < PH; ++i)
+            for (int j = 0; j < PW; ++j) {
+                const float *d = offset + (((size_t)n * PH + i) * PW + j) * 2;
+                const float dx = (gamma * d[0]) * rw, dy = (gamma * d[1]) * rh;
+                const float bx0 = x1 + (float)j * bw, by0 = y1 + (float)i * bh;
+                double *y = out + (((size_t)n * PH + i) * PW + j) * C;
+                for (int c = 0; c < C; ++c) y[c] = 0.0;
+                int not_a_number = 0;
+                for (int sy = 0; sy < S; ++sy)
+                    for (int sx = 0; sx < S; ++sx) {
+                        const float py = (by0 + ((float)sy + 0.5f) * sh) + dy;
+                        const float px = (bx0 + ((float)sx + 0.5f) * sw) + dx;
+                        if (isnan(px) || isnan(py)) { not_a_number = 1; continue; }
+                        const double fy = floor((double)py), fx = floor((double)px);
+                        if (!(fy >= -1.0 && fy <= H - 1 && fx >= -1.0 && fx <= W - 1)) continue;
+                        const int y0 = (int)fy, x0 = (int)fx;
+                        for (int qy = y0; qy <= y0 + 1; ++qy) {
+                            if (qy < 0 || qy >= H) continue;
+                            const double gy = g_kernel(qy, py);
+                            for (int qx = x0; qx <= x0 + 1; ++qx) {
+                                if (qx < 0 || qx >= W) continue;
+                                const double Gq = g_kernel(qx, px) * gy;
+                                const double *xq = x + (((size_t)b * H + qy) * W + qx) * (size_t)C;
+                                for (int c = 0; c < C; ++c) y[c] += Gq * xq[c];
+                            }
+                        }
+                    }
+                for (int c = 0; c < C; ++c) y[c] = not_a_number ? NAN : y[c] / (double)(S * S);
+            }
+    }
+    (void)B;
+}

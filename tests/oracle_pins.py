@@ -448,3 +448,102 @@ CORE_PINS = [pin_identity, pin_box_sum, pin_shifted_gather, pin_affine_field, pi
 BACKWARD_PINS = [pin_backward_fd, pin_backward_autograd]
 AGG_PINS = [pin_agg_brute_force, pin_agg_grid_sample, pin_agg_backward]
 ALL_PINS = CORE_PINS + BACKWARD_PINS + AGG_PINS
+
+
+# ---------------------------------------------------------------- deformable RoI pooling pins
+def roi_case(seed, B=2, H=13, W=17, C=3, N=6, P=(3, 4), scale=0.5, margin=2.0, off_std=0.5, quant=None):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B, H, W, C))
+    rois = []
+    for n in range(N):
+        b = n % B
+        w_img, h_img = W / scale, H / scale
+        x1 = rng.uniform(margin / scale, w_img / 2)
+        y1 = rng.uniform(margin / scale, h_img / 2)
+        x2 = rng.uniform(x1 + 1.0, w_img - margin / scale)
+        y2 = rng.uniform(y1 + 1.0, h_img - margin / scale)
+        rois.append([b, x1, y1, x2, y2])
+    rois = np.array(rois, dtype=np.float32)
+    off = (rng.standard_normal((N, P[0], P[1], 2)) * off_std).astype(np.float32)
+    if quant is not None:
+        off = (np.round(off / quant) * quant).astype(np.float32)
+    return x, rois, off
+
+
+def roi_positions32(rois, off, P, S, scale, gamma):
+    """fp32 sample positions py, px [N, PH, PW, S, S] in the oracle's operation order."""
+    f = np.float32
+    r = rois.astype(f)
+    x1, y1, x2, y2 = r[:, 1] * f(scale), r[:, 2] * f(scale), r[:, 3] * f(scale), r[:, 4] * f(scale)
+    rw = np.maximum(x2 - x1, f(1)).astype(f)
+    rh = np.maximum(y2 - y1, f(1)).astype(f)
+    bw, bh = (rw / f(P[1])).astype(f), (rh / f(P[0])).astype(f)
+    sw, sh = (bw / f(S)).astype(f), (bh / f(S)).astype(f)
+    i = np.arange(P[0], dtype=f)[None, :, None, None, None]
+    j = np.arange(P[1], dtype=f)[None, None, :, None, None]
+    sy = (np.arange(S, dtype=f) + f(0.5))[None, None, None, :, None]
+    sx = (np.arange(S, dtype=f) + f(0.5))[None, None, None, None, :]
+    dx = ((f(gamma) * off[..., 0]).astype(f) * rw[:, None, None]).astype(f)[..., None, None]
+    dy = ((f(gamma) * off[..., 1]).astype(f) * rh[:, None, None]).astype(f)[..., None, None]
+    by0 = (y1[:, None, None, None, None] + (i * bh[:, None, None, None, None]).astype(f)).astype(f)
+    bx0 = (x1[:, None, None, None, None] + (j * bw[:, None, None, None, None]).astype(f)).astype(f)
+    py = ((by0 + (sy * sh[:, None, None, None, None]).astype(f)).astype(f) + dy).astype(f)
+    px = ((bx0 + (sx * sw[:, None, None, None, None]).astype(f)).astype(f) + dx).astype(f)
+    return py.astype(np.float64), px.astype(np.float64)
+
+
+def pin_roi_brute_force(lib):
+    """Average over S x S samples of the sum over every grid point of G(q,p) x(q)."""
+    for seed, (P, S, scale, gamma) in enumerate((((3, 4), 2, 0.5, 0.1), ((2, 2), 3, 1.0, 0.3),
+                                                 ((5, 3), 1, 0.25, 1.0))):
+        x, rois, off = roi_case(80 + seed, P=P, scale=scale, margin=-1.0, off_std=2.0)
+        out = oracle.roi_pool_forward(x, rois, off, pooled=P, sampling=S, spatial_scale=scale, gamma=gamma,
+                                      lib=lib)
+        py, px = roi_positions32(rois, off, P, S, scale, gamma)
+        B, H, W, C = x.shape
+        gy = np.maximum(0, 1 - np.abs(np.arange(H) - py[..., None]))
+        gx = np.maximum(0, 1 - np.abs(np.arange(W) - px[..., None]))
+        xb = x[rois[:, 0].astype(int)]  # [N, H, W, C]
+        ref = np.einsum("nijabh,nijabw,nhwc->nijc", gy, gx, xb) / (S * S)
+        assert np.allclose(out, ref, rtol=0, atol=1e-12), "roi brute force"
+
+
+def pin_roi_affine(lib):
+    """On x = a + b*y + c*x the pooled value is the field at the mean sample position."""
+    rng = np.random.default_rng(90)
+    B, H, W, C = 2, 20, 24, 3
+    a, bcoef, ccoef = rng.standard_normal((3, C))
+    yy, xx = np.meshgrid(np.arange(H), np.arange(W), indexing="ij")
+    x = np.broadcast_to(a + bcoef * yy[..., None] + ccoef * xx[..., None], (B, H, W, C)).copy()
+    _, rois, off = roi_case(91, B=B, H=H, W=W, C=C, N=8, P=(3, 2), scale=0.5, margin=5.0, off_std=0.3)
+    out = oracle.roi_pool_forward(x, rois, off, pooled=(3, 2), sampling=2, spatial_scale=0.5, gamma=0.2,
+                                  lib=lib)
+    py, px = roi_positions32(rois, off, (3, 2), 2, 0.5, 0.2)
+    assert (py >= 0).all() and (py <= H - 1).all() and (px >= 0).all() and (px <= W - 1).all()
+    my, mx = py.mean(axis=(-1, -2)), px.mean(axis=(-1, -2))
+    ref = a + bcoef * my[..., None] + ccoef * mx[..., None]
+    assert np.allclose(out, ref, rtol=0, atol=1e-11), "roi affine"
+
+
+def pin_roi_constant(lib):
+    x = np.full((1, 9, 9, 2), -2.5)
+    _, rois, off = roi_case(92, B=1, H=9, W=9, C=2, N=5, P=(2, 2), scale=1.0, margin=2.5, off_std=0.1)
+    out = oracle.roi_pool_forward(x, rois, off, pooled=(2, 2), sampling=2, spatial_scale=1.0, gamma=0.1, lib=lib)
+    assert np.allclose(out, -2.5, rtol=0, atol=1e-13), "roi constant"
+
+
+def pin_roi_torchvision(lib):
+    """Zero offsets reduce to RoIAlign (torchvision, aligned=False) for regions inside the map."""
+    import torchvision
+
+    x, rois, off = roi_case(93, B=2, H=21, W=19, C=4, N=10, P=(4, 3), scale=0.5, margin=3.0)
+    off[:] = 0
+    out = oracle.roi_pool_forward(x, rois, off, pooled=(4, 3), sampling=2, spatial_scale=0.5, gamma=0.1, lib=lib)
+    ref = torchvision.ops.roi_align(torch.from_numpy(x).permute(0, 3, 1, 2).contiguous(),
+                                    torch.from_numpy(rois.astype(np.float64)), output_size=(4, 3),
+                                    spatial_scale=0.5, sampling_ratio=2, aligned=False)
+    assert np.allclose(out, ref.permute(0, 2, 3, 1).numpy(), rtol=0, atol=1e-5), "roi torchvision"
+
+
+ROI_PINS = [pin_roi_brute_force, pin_roi_affine, pin_roi_constant, pin_roi_torchvision]
+ALL_PINS = ALL_PINS + ROI_PINS

@@ -95,6 +95,17 @@ MUTATIONS = [
     ("glp[li + 0] += w * dpx * Ws;", "glp[li + 0] += w * dpx;", 0, pins.AGG_PINS),
     ("grad_feat[off + c] += w * gx * gy * go[c];", "grad_feat[off + c] += gx * gy * go[c];", 0,
      pins.AGG_PINS),
+    ("const float dx = (gamma * d[0]) * rw, dy = (gamma * d[1]) * rh;",
+     "const float dx = (gamma * d[1]) * rw, dy = (gamma * d[0]) * rh;", 0, pins.ROI_PINS),
+    ("const float dx = (gamma * d[0]) * rw, dy = (gamma * d[1]) * rh;",
+     "const float dx = (gamma * d[0]) * rw, dy = (gamma * d[1]) * rw;", 0, pins.ROI_PINS),
+    ("const float bx0 = x1 + (float)j * bw, by0 = y1 + (float)i * bh;",
+     "const float bx0 = x1 + (float)i * bw, by0 = y1 + (float)j * bh;", 0, pins.ROI_PINS),
+    ("y[c] / (double)(S * S)", "y[c] / (double)S", 0, pins.ROI_PINS),
+    ("const float px = (bx0 + ((float)sx + 0.5f) * sw) + dx;", "const float px = (bx0 + (float)sx * sw) + dx;", 0,
+     pins.ROI_PINS),
+    ("const float x1 = r[1] * spatial_scale, y1 = r[2] * spatial_scale;",
+     "const float x1 = r[1], y1 = r[2] * spatial_scale;", 0, pins.ROI_PINS),
 ]
 
 
