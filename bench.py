@@ -321,7 +321,7 @@ def measure_rows(dcn, dev, stream, l2, barrier, world, steps=280):
     def core_fwd(name):
         shape, inp = si.workload_core(name)
         x, off, m = (inp[k].to(dev) for k in ("x", "offset", "mask"))
-        R = max(2, math.ceil(4 * l2 / shape.compulsory_bytes()))
+        R = min(64, max(2, math.ceil(4 * l2 / shape.compulsory_bytes())))
         sets = [(x.clone(), off.clone(), m.clone(),
                  torch.empty((shape.B, shape.Ho, shape.Wo, shape.G * shape.C), dtype=x.dtype, device=dev))
                 for _ in range(R)]
@@ -338,6 +338,24 @@ def measure_rows(dcn, dev, stream, l2, barrier, world, steps=280):
 
     for n in ("dcnv3_tiny", "dcnv3_p3", "dcnv3_p3_dil2"):
         core_fwd(n)
+
+    # DCNv3 softmax-mode backward, bf16, at the P3 shape
+    shape, inp = si.workload_core("dcnv3_p3")
+    g = torch.from_numpy(__import__("numpy").random.default_rng(6).standard_normal(
+        (shape.B, shape.Ho, shape.Wo, shape.G * shape.C))).to(torch.bfloat16)
+    t = [inp[k].to(dev) for k in ("x", "offset", "mask")] + [g.to(dev)]
+    R = max(2, math.ceil(4 * l2 / shape.compulsory_bytes(backward=True)))
+    sets = [[u.clone() for u in t] + [torch.empty_like(t[0]), torch.empty_like(t[1]), torch.empty_like(t[2])]
+            for _ in range(R)]
+
+    def mkb3(s):
+        return lambda: dcn.dcn_core_backward(s[0], s[1], s[2], s[3], group=shape.G, softmax=True, grad_x=s[4],
+                                             grad_offset=s[5], grad_mask=s[6])
+
+    ms = time_steps(mkb3, sets, steps, 3 * R, stream, barrier, world) / steps
+    out["dcnv3_p3_bwd_softmax_bf16"] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(shape.samples / ms / 1e6, 2),
+                                        "R": R}
+    del sets
 
     # DCNv4 backward at the P4 shape, fp32
     shape, inp = si.workload_core("dcnv4_p4_bwd")
@@ -369,6 +387,36 @@ def measure_rows(dcn, dev, stream, l2, barrier, world, steps=280):
     ms = time_steps(mka, sets, steps, 3 * R, stream, barrier, world) / steps
     out["sparse4d"] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(a.samples / ms / 1e6, 2),
                        "GB_s": round(a.compulsory_bytes() / ms / 1e6, 1), "R": R}
+    del sets
+
+    # Sparse4D aggregation backward
+    inp = si.agg_inputs(a, si.SEEDS["sparse4d"], with_grad_out=True)
+    t = [inp[k].to(dev) for k in keys + ("grad_out",)]
+    R = max(2, math.ceil(4 * l2 / (2 * a.compulsory_bytes())))
+    sets = [[u.clone() for u in t] + [torch.empty_like(t[0]), torch.empty_like(t[3]), torch.empty_like(t[4])]
+            for _ in range(R)]
+
+    def mkab(s):
+        return lambda: dcn.deform_agg_backward(*s[:6], grad_feat=s[6], grad_loc=s[7], grad_weights=s[8])
+
+    ms = time_steps(mkab, sets, steps, 3 * R, stream, barrier, world) / steps
+    out["sparse4d_bwd"] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(a.samples / ms / 1e6, 2), "R": R}
+    del sets
+
+    # deformable RoI pooling
+    rs = si.ROI_POOL
+    inp = si.roi_inputs(rs, si.SEEDS["roi_pool"])
+    t = [inp[k].to(dev) for k in ("x", "rois", "offset")]
+    R = max(2, math.ceil(4 * l2 / rs.compulsory_bytes()))
+    sets = [[u.clone() for u in t] + [torch.empty((rs.N, rs.PH, rs.PW, rs.C), device=dev)] for _ in range(R)]
+
+    def mkr(s):
+        return lambda: dcn.deform_roi_pool_forward(s[0], s[1], s[2], pooled=(rs.PH, rs.PW), sampling=rs.S,
+                                                   spatial_scale=rs.spatial_scale, gamma=rs.gamma, out=s[3])
+
+    ms = time_steps(mkr, sets, steps, 3 * R, stream, barrier, world) / steps
+    out["roi_pool"] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(rs.samples / ms / 1e6, 2),
+                       "GB_s": round(rs.compulsory_bytes() / ms / 1e6, 1), "R": R}
     return out
 
 

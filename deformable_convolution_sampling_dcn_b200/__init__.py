@@ -4,6 +4,7 @@ Thin Python front end of libdcn_b200.so (C ABI in include/dcn_b200.h):
 
     dcn_core_forward / dcn_core_backward     DCNv2/v3/v4 sampling core
     deform_agg_forward / deform_agg_backward Sparse4D multi-camera aggregation
+    deform_roi_pool_forward                  deformable RoI pooling
     DCNCoreFunction, DeformAggFunction       autograd wrappers over the above
     shard_range                              batch split for one-process-per-GPU runs
 
@@ -16,11 +17,12 @@ from typing import Tuple
 
 import torch
 
-from ._binding import (ABI_VERSION, EXPORTS, DaggParams, DcnError, DcnParams, core_params, dcn_core_backward,
-                       dcn_core_forward, dcn_core_output_hw, deform_agg_backward, deform_agg_forward, lib)
+from ._binding import (ABI_VERSION, EXPORTS, DaggParams, DcnError, DcnParams, DroiParams, core_params,
+                       dcn_core_backward, dcn_core_forward, dcn_core_output_hw, deform_agg_backward,
+                       deform_agg_forward, deform_roi_pool_forward, lib)
 
 __all__ = ["dcn_core_forward", "dcn_core_backward", "dcn_core_output_hw", "deform_agg_forward",
-           "deform_agg_backward", "DCNCoreFunction", "DeformAggFunction", "shard_range", "lib", "DcnError",
+           "deform_agg_backward", "deform_roi_pool_forward", "DroiParams", "DCNCoreFunction", "DeformAggFunction", "shard_range", "lib", "DcnError",
            "DcnParams", "DaggParams", "core_params", "EXPORTS", "ABI_VERSION"]
 
 

@@ -26,7 +26,7 @@ _DTYPE_CODE = {torch.float32: DCN_F32, torch.float16: DCN_F16, torch.bfloat16: D
 # Every entry point include/dcn_b200.h declares.
 EXPORTS = ("dcn_core_output_hw", "dcn_core_forward", "dcn_core_backward", "deform_agg_forward",
            "deform_agg_backward", "dcn_status_string", "dcn_last_error_detail", "dcn_abi_version",
-           "dcn_take_device_error")
+           "dcn_take_device_error", "deform_roi_pool_forward")
 ABI_VERSION = 1
 
 
@@ -39,6 +39,12 @@ class DcnParams(ctypes.Structure):
 class DaggParams(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("B", "num_cams", "num_scales", "num_rows", "num_anchors",
                                               "num_pts", "G", "C", "dtype")]
+
+
+class DroiParams(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "H", "W", "C", "num_rois", "pooled_h", "pooled_w",
+                                              "sampling")] + \
+               [("spatial_scale", ctypes.c_float), ("gamma", ctypes.c_float), ("dtype", ctypes.c_int32)]
 
 
 class DcnError(RuntimeError):
@@ -70,6 +76,8 @@ def _declare(lib):
     lib.dcn_last_error_detail.restype = ctypes.c_char_p
     lib.dcn_abi_version.argtypes = []
     lib.dcn_abi_version.restype = ctypes.c_int32
+    lib.deform_roi_pool_forward.argtypes = [ctypes.POINTER(DroiParams), vp, vp, vp, vp, vp]
+    lib.deform_roi_pool_forward.restype = st
     lib.dcn_take_device_error.argtypes = []
     lib.dcn_take_device_error.restype = ctypes.c_int32
     return lib
@@ -250,3 +258,26 @@ def deform_agg_backward(feat, spatial_shape, scale_start_index, sampling_locatio
                                     weights.data_ptr(), grad_out.data_ptr(), grad_feat.data_ptr(),
                                     grad_loc.data_ptr(), grad_weights.data_ptr(), _stream(feat)))
     return grad_feat, grad_loc, grad_weights
+
+
+def deform_roi_pool_forward(x, rois, offset, *, pooled=(7, 7), sampling: int = 2, spatial_scale: float = 1.0,
+                            gamma: float = 0.1, out=None):
+    """out [N, PH, PW, C]: deformable RoI pooling of x [B, H, W, C]; see dcn_b200.h."""
+    _cuda_tensor("x", x)
+    if x.dtype not in _DTYPE_CODE:
+        raise TypeError(f"unsupported dtype {x.dtype}")
+    _cuda_tensor("rois", rois, torch.float32)
+    _cuda_tensor("offset", offset, torch.float32)
+    B, H, W, C = x.shape
+    PH, PW = _pair(pooled)
+    N = rois.shape[0]
+    if tuple(rois.shape) != (N, 5) or tuple(offset.shape) != (N, PH, PW, 2):
+        raise ValueError("rois must be [N, 5] and offset [N, PH, PW, 2]")
+    p = DroiParams(B, H, W, C, N, PH, PW, int(sampling), float(spatial_scale), float(gamma), _DTYPE_CODE[x.dtype])
+    if out is None:
+        out = torch.empty((N, PH, PW, C), dtype=x.dtype, device=x.device)
+    else:
+        _cuda_tensor("out", out, x.dtype)
+    check(lib().deform_roi_pool_forward(ctypes.byref(p), x.data_ptr(), rois.data_ptr(), offset.data_ptr(),
+                                        out.data_ptr(), _stream(x)))
+    return out

@@ -197,6 +197,34 @@ dcn_status deform_agg_forward(const dagg_params *p, const void *feat, const int3
     return cuda_status(dcnb::launch_agg_forward(a, (cudaStream_t)stream), "deform_agg_forward launch");
 }
 
+dcn_status deform_roi_pool_forward(const droi_params *p, const void *x, const float *rois, const float *offset,
+                                   void *out, dcn_stream_t stream) {
+    if (!p) return fail(DCN_ERR_NULL, "params is NULL");
+    if (p->dtype < DCN_F32 || p->dtype > DCN_BF16) return fail(DCN_ERR_UNSUPPORTED, "dtype %d", p->dtype);
+    if (p->B < 1 || p->H < 1 || p->W < 1 || p->C < 1 || p->num_rois < 0 || p->pooled_h < 1 || p->pooled_w < 1 ||
+        p->sampling < 1)
+        return fail(DCN_ERR_SHAPE, "sizes must be positive (num_rois may be 0)");
+    if (p->B > kMaxDim || p->H > kMaxDim || p->W > kMaxDim || p->C > 65536 || p->pooled_h > 1024 ||
+        p->pooled_w > 1024 || p->sampling > 64 || p->num_rois > (1 << 24))
+        return fail(DCN_ERR_SHAPE, "a size exceeds its limit");
+    if (!isfinite(p->spatial_scale) || !isfinite(p->gamma)) return fail(DCN_ERR_SHAPE, "scale/gamma not finite");
+    if ((long long)p->num_rois * p->pooled_h * p->pooled_w > (1LL << 31))
+        return fail(DCN_ERR_SHAPE, "num_rois * pooled_h * pooled_w exceeds 2^31");
+    if (((size_t)p->C * dtype_size(p->dtype)) % 16 != 0)
+        return fail(DCN_ERR_UNSUPPORTED, "C*sizeof(dtype) must be a multiple of 16 bytes");
+    if (p->num_rois == 0) return DCN_OK;
+    if (!x || !rois || !offset || !out) return fail(DCN_ERR_NULL, "x, rois, offset and out are required");
+    if (!aligned(x, 16) || !aligned(out, 16)) return fail(DCN_ERR_ALIGN, "x and out must be 16-byte aligned");
+    if (!aligned(rois, 4) || !aligned(offset, 8)) return fail(DCN_ERR_ALIGN, "rois 4-byte, offset 8-byte alignment");
+    dcnb::RoiArgs a;
+    a.x = x; a.rois = rois; a.offset = offset; a.out = out;
+    a.B = p->B; a.H = p->H; a.W = p->W; a.C = p->C; a.N = p->num_rois;
+    a.PH = p->pooled_h; a.PW = p->pooled_w; a.S = p->sampling;
+    a.spatial_scale = p->spatial_scale; a.gamma = p->gamma;
+    a.dtype = (dcnb::DType)p->dtype;
+    return cuda_status(dcnb::launch_roi_pool_forward(a, (cudaStream_t)stream), "deform_roi_pool_forward launch");
+}
+
 dcn_status deform_agg_backward(const dagg_params *p, const void *feat, const int32_t *spatial_shape,
                                const int32_t *scale_start_index, const float *sampling_location,
                                const void *weights, const void *grad_out, void *grad_feat, float *grad_loc,

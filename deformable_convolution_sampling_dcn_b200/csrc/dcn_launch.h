@@ -42,6 +42,16 @@ struct AggArgs {
     DType dtype;
 };
 
+struct RoiArgs {
+    const void *x;       // [B, H, W, C]
+    const float *rois;   // [N, 5]
+    const float *offset; // [N, PH, PW, 2]
+    void *out;           // [N, PH, PW, C]
+    int B, H, W, C, N, PH, PW, S;
+    float spatial_scale, gamma;
+    DType dtype;
+};
+
 // Each launcher enqueues its kernel(s) on `stream` and returns the
 // cudaGetLastError() of the launch.
 cudaError_t launch_core_forward_generic(const CoreArgs &a, cudaStream_t stream);
@@ -57,5 +67,6 @@ cudaError_t launch_agg_forward(const AggArgs &a, cudaStream_t stream);
 // (and launches nothing) when the feature row width does not fit them.
 cudaError_t launch_agg_wide(const AggArgs &a, bool bwd, cudaStream_t stream, bool *handled);
 cudaError_t launch_agg_backward(const AggArgs &a, cudaStream_t stream);
+cudaError_t launch_roi_pool_forward(const RoiArgs &a, cudaStream_t stream);
 
 }  // namespace dcnb

@@ -1,0 +1,109 @@
+// Deformable RoI pooling, forward ("用PyTorch实战DCNv1：从零构建可变形卷积与ROI池化模块",
+// section 3): each of the PH x PW bins of a region of interest is moved by
+// dp = gamma * dp_hat o (w, h), the learned offset normalised by the region
+// size, and averages S x S bilinear samples of the NHWC map (the bilinear
+// kernel of section 2, zeros outside the map).
+//
+// One warp per (roi, bin); lanes own 16-byte channel chunks, so each corner
+// read is a coalesced C-contiguous row.  The sample positions are formed in
+// fp32 with one rounding per operation in a fixed order (no contraction),
+// so the floor() decisions are reproducible.
+#include "dcn_common.cuh"
+#include "dcn_launch.h"
+
+namespace dcnb {
+namespace {
+
+template <typename T>
+__global__ void __launch_bounds__(256) roi_pool_forward_kernel(RoiArgs a) {
+    constexpr int V = Storage<T>::kVec;
+    const int lane = threadIdx.x & 31;
+    const long long bins = (long long)a.N * a.PH * a.PW;
+    const long long bin = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (bin >= bins) return;
+    const int j = (int)(bin % a.PW);
+    const int i = (int)((bin / a.PW) % a.PH);
+    const long long n = bin / ((long long)a.PW * a.PH);
+    const float *r = a.rois + n * 5;
+    const float rb = __ldg(r);
+    const int b = (int)rb;
+    const int chunks = a.C / V;
+    T *o = static_cast<T *>(a.out) + bin * a.C;
+    if (!(rb >= 0.0f && rb < (float)a.B)) {  // batch index outside the input: nothing to read
+        for (int c = lane; c < chunks; c += 32) {
+            float z[V];
+#pragma unroll
+            for (int v = 0; v < V; ++v) z[v] = 0.0f;
+            *reinterpret_cast<uint4 *>(o + c * V) = pack16<T>(z);
+        }
+        return;
+    }
+    const float x1 = __fmul_rn(__ldg(r + 1), a.spatial_scale), y1 = __fmul_rn(__ldg(r + 2), a.spatial_scale);
+    const float x2 = __fmul_rn(__ldg(r + 3), a.spatial_scale), y2 = __fmul_rn(__ldg(r + 4), a.spatial_scale);
+    float rw = __fsub_rn(x2, x1), rh = __fsub_rn(y2, y1);
+    if (!(rw >= 1.0f)) rw = 1.0f;
+    if (!(rh >= 1.0f)) rh = 1.0f;
+    const float bw = __fdiv_rn(rw, (float)a.PW), bh = __fdiv_rn(rh, (float)a.PH);
+    const float sw = __fdiv_rn(bw, (float)a.S), sh = __fdiv_rn(bh, (float)a.S);
+    const float2 d = __ldg(reinterpret_cast<const float2 *>(a.offset) + bin);
+    const float dx = __fmul_rn(__fmul_rn(a.gamma, d.x), rw), dy = __fmul_rn(__fmul_rn(a.gamma, d.y), rh);
+    const float bx0 = __fadd_rn(x1, __fmul_rn((float)j, bw)), by0 = __fadd_rn(y1, __fmul_rn((float)i, bh));
+    const T *xb = static_cast<const T *>(a.x) + (long long)b * a.H * a.W * a.C;
+    const float inv = 1.0f / (float)(a.S * a.S);
+
+    for (int c = lane; c < chunks; c += 32) {
+        float acc[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = 0.0f;
+        bool nan_pos = false;
+        for (int sy = 0; sy < a.S; ++sy) {
+            const float py = __fadd_rn(__fadd_rn(by0, __fmul_rn((float)sy + 0.5f, sh)), dy);
+            for (int sx = 0; sx < a.S; ++sx) {
+                const float px = __fadd_rn(__fadd_rn(bx0, __fmul_rn((float)sx + 0.5f, sw)), dx);
+                Tap tp{0, 0, 0.0f, 0.0f};
+                const int st = make_tap(py, px, a.H, a.W, tp);
+                if (st < 0) nan_pos = true;
+                if (st <= 0) continue;
+                const float gyv[2] = {1.0f - tp.ly, tp.ly};
+                const float gxv[2] = {1.0f - tp.lx, tp.lx};
+#pragma unroll
+                for (int cy = 0; cy < 2; ++cy) {
+#pragma unroll
+                    for (int cx = 0; cx < 2; ++cx) {
+                        const int y = tp.y0 + cy, x = tp.x0 + cx;
+                        if (y < 0 || y >= a.H || x < 0 || x >= a.W) continue;
+                        float f[V];
+                        unpack16<T>(ld_nc16(xb + ((long long)y * a.W + x) * a.C + c * V), f);
+                        const float g = gyv[cy] * gxv[cx];
+#pragma unroll
+                        for (int v = 0; v < V; ++v) acc[v] = fmaf(g, f[v], acc[v]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = nan_pos ? __int_as_float(0x7fc00000) : acc[v] * inv;
+        *reinterpret_cast<uint4 *>(o + c * V) = pack16<T>(acc);
+    }
+}
+
+template <typename T>
+cudaError_t launch_t(const RoiArgs &a, cudaStream_t stream) {
+    const long long bins = (long long)a.N * a.PH * a.PW;
+    const long long blocks = (bins + 7) / 8;
+    roi_pool_forward_kernel<T><<<(unsigned)blocks, 256, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_roi_pool_forward(const RoiArgs &a, cudaStream_t stream) {
+    switch (a.dtype) {
+        case DType::F32: return launch_t<float>(a, stream);
+        case DType::F16: return launch_t<__half>(a, stream);
+        case DType::BF16: return launch_t<__nv_bfloat16>(a, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace dcnb

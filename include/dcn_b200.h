@@ -165,6 +165,36 @@ dcn_status deform_agg_backward(const dagg_params *p, const void *feat,
                                const void *grad_out, void *grad_feat, float *grad_loc,
                                void *grad_weights, dcn_stream_t stream);
 
+/*
+ * Deformable RoI pooling, forward ("用PyTorch实战DCNv1：从零构建可变形卷积与ROI池化模块",
+ * section 3): bin (i, j) of region n is moved by
+ * dp = gamma * dp_hat o (w, h) (the offset normalised by the region's width and
+ * height) and averages S x S bilinear samples (zeros outside the map).
+ *   x      [B, H, W, C]          NHWC, storage dtype
+ *   rois   [N, 5] fp32           (batch index, x1, y1, x2, y2) in input-image units,
+ *                                scaled by spatial_scale; a batch index outside
+ *                                [0, B) reads nothing and yields zeros
+ *   offset [N, PH, PW, 2] fp32   (dx_hat, dy_hat)
+ *   out    [N, PH, PW, C]        storage dtype
+ * Region size max(x2 - x1, 1) x max(y2 - y1, 1) after scaling; bin (i, j)
+ * starts at (x1 + j*w/PW, y1 + i*h/PH); sample (sy, sx) sits at
+ * + ((s + 0.5) * bin / S) + dp, pixel centres at integers; positions are
+ * formed in fp32, one rounding per operation in that order.  A NaN position
+ * makes its bin NaN.  C*sizeof(dtype) must be a multiple of 16 bytes (at most
+ * 65536 channels); x and out 16-byte aligned, rois/offset 8-byte aligned.
+ */
+typedef struct {
+    int32_t B, H, W, C;           /* input map */
+    int32_t num_rois;             /* N */
+    int32_t pooled_h, pooled_w;   /* PH, PW */
+    int32_t sampling;             /* S >= 1 samples per bin side */
+    float spatial_scale, gamma;
+    int32_t dtype;                /* dcn_dtype */
+} droi_params;
+
+dcn_status deform_roi_pool_forward(const droi_params *p, const void *x, const float *rois,
+                                   const float *offset, void *out, dcn_stream_t stream);
+
 /* Static, human-readable name of a status. */
 const char *dcn_status_string(dcn_status s);
 

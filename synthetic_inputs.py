@@ -246,3 +246,55 @@ def agg_inputs(shape: AggShape, seed: int, *, with_grad_out: bool = False,
         out["grad_out"] = _round(rng.standard_normal((s.B, s.num_anchors, s.G * s.C)), s.dtype)
     return out
 
+
+
+@dataclasses.dataclass(frozen=True)
+class RoiShape:
+    """Shape of one deformable RoI pooling problem."""
+
+    B: int
+    H: int
+    W: int
+    C: int
+    N: int
+    PH: int = 7
+    PW: int = 7
+    S: int = 2
+    spatial_scale: float = 1.0 / 16
+    gamma: float = 0.1
+    dtype: str = "f32"
+
+    @property
+    def samples(self) -> int:
+        return self.N * self.PH * self.PW * self.S * self.S
+
+    def compulsory_bytes(self) -> int:
+        e = torch.finfo(DTYPES[self.dtype]).bits // 8
+        return (self.B * self.H * self.W * self.C * e + self.N * 5 * 4 + self.N * self.PH * self.PW * 2 * 4
+                + self.N * self.PH * self.PW * self.C * e)
+
+
+# Deformable RoI pooling on a stride-16 feature map of a 1024 x 1024 image:
+# 512 regions, 7 x 7 bins, 2 x 2 samples per bin, 256 channels.
+ROI_POOL = RoiShape(B=2, H=64, W=64, C=256, N=512)
+SEEDS["roi_pool"] = 5
+
+
+def roi_inputs(shape: RoiShape, seed: int, *, offset_std: float = 1.0,
+               min_size: float = 16.0) -> Dict[str, torch.Tensor]:
+    """x [B,H,W,C] ~ N(0,1); rois [N,5] with boxes uniform inside the image
+    (W/spatial_scale x H/spatial_scale, at least min_size wide); offset
+    [N,PH,PW,2] ~ N(0, offset_std) (normalised units)."""
+    s = shape
+    rng = np.random.Generator(np.random.PCG64(seed))
+    x = rng.standard_normal((s.B, s.H, s.W, s.C))
+    img_w, img_h = s.W / s.spatial_scale, s.H / s.spatial_scale
+    b = rng.integers(0, s.B, s.N)
+    x1 = rng.uniform(0, img_w - min_size, s.N)
+    y1 = rng.uniform(0, img_h - min_size, s.N)
+    x2 = np.minimum(x1 + min_size + rng.exponential(img_w / 6, s.N), img_w)
+    y2 = np.minimum(y1 + min_size + rng.exponential(img_h / 6, s.N), img_h)
+    rois = np.stack([b, x1, y1, x2, y2], axis=1).astype(np.float32)
+    off = rng.standard_normal((s.N, s.PH, s.PW, 2)) * offset_std
+    return {"x": _round(x, s.dtype), "rois": torch.from_numpy(rois),
+            "offset": torch.from_numpy(off.astype(np.float32))}

@@ -132,3 +132,16 @@ def test_shard_range():
             assert all(parts[i][1] == parts[i + 1][0] for i in range(world - 1))
             sizes = [hi - lo for lo, hi in parts]
             assert max(sizes) - min(sizes) <= 1
+
+
+def test_roi_pool_checks(lib):
+    p = B.DroiParams(2, 64, 64, 256, 10, 7, 7, 2, 0.0625, 0.1, 0)
+    assert lib.deform_roi_pool_forward(ctypes.byref(p), 16, 16, 16, 0, None) == B.DCN_ERR_NULL
+    assert lib.deform_roi_pool_forward(ctypes.byref(p), 8, 16, 16, 16, None) == B.DCN_ERR_ALIGN
+    assert lib.deform_roi_pool_forward(ctypes.byref(p), 16, 16, 12, 16, None) == B.DCN_ERR_ALIGN
+    bad = B.DroiParams(2, 64, 64, 6, 10, 7, 7, 2, 0.0625, 0.1, 1)  # 12-byte rows
+    assert lib.deform_roi_pool_forward(ctypes.byref(bad), 16, 16, 16, 16, None) == B.DCN_ERR_UNSUPPORTED
+    bad = B.DroiParams(2, 64, 64, 256, 10, 7, 7, 0, 0.0625, 0.1, 0)
+    assert lib.deform_roi_pool_forward(ctypes.byref(bad), 16, 16, 16, 16, None) == B.DCN_ERR_SHAPE
+    empty = B.DroiParams(2, 64, 64, 256, 0, 7, 7, 2, 0.0625, 0.1, 0)
+    assert lib.deform_roi_pool_forward(ctypes.byref(empty), None, None, None, None, None) == B.DCN_OK

@@ -1,0 +1,59 @@
+"""GPU parity of deform_roi_pool_forward against the fp64 oracle."""
+import pytest
+import torch
+
+import oracle
+import synthetic_inputs as si
+from parity import assert_close_fwd
+
+pytestmark = pytest.mark.gpu
+
+
+def run(shape: si.RoiShape, inp, dev):
+    import deformable_convolution_sampling_dcn_b200 as d
+
+    out = d.deform_roi_pool_forward(inp["x"].to(dev), inp["rois"].to(dev), inp["offset"].to(dev),
+                                    pooled=(shape.PH, shape.PW), sampling=shape.S,
+                                    spatial_scale=shape.spatial_scale, gamma=shape.gamma)
+    torch.cuda.synchronize()
+    ref = oracle.roi_pool_forward(inp["x"], inp["rois"], inp["offset"], pooled=(shape.PH, shape.PW),
+                                  sampling=shape.S, spatial_scale=shape.spatial_scale, gamma=shape.gamma)
+    return out, ref
+
+
+def test_roi_pool_workload(cuda_dev):
+    shape = si.ROI_POOL
+    inp = si.roi_inputs(shape, si.SEEDS["roi_pool"])
+    out, ref = run(shape, inp, cuda_dev)
+    assert_close_fwd(out, ref, "roi pool")
+
+
+@pytest.mark.parametrize("case", [
+    # B, H, W, C, N, PH, PW, S, scale, gamma, dtype
+    (1, 9, 13, 8, 5, 3, 4, 2, 0.5, 0.1, "f32"),
+    (2, 20, 17, 64, 33, 7, 7, 3, 0.25, 0.3, "f16"),
+    (3, 11, 11, 16, 7, 2, 5, 1, 1.0, 1.0, "bf16"),
+    (1, 33, 40, 512, 9, 4, 4, 2, 0.125, 0.2, "f16"),
+])
+def test_roi_pool_small(case, cuda_dev):
+    B, H, W, C, N, PH, PW, S, sc, gm, dt = case
+    shape = si.RoiShape(B=B, H=H, W=W, C=C, N=N, PH=PH, PW=PW, S=S, spatial_scale=sc, gamma=gm, dtype=dt)
+    inp = si.roi_inputs(shape, 500 + N, offset_std=1.5, min_size=2.0)
+    out, ref = run(shape, inp, cuda_dev)
+    assert_close_fwd(out, ref, f"roi small {case}")
+
+
+def test_roi_bad_batch_index_reads_nothing(cuda_dev):
+    import deformable_convolution_sampling_dcn_b200 as d
+
+    shape = si.RoiShape(B=1, H=8, W=8, C=32, N=3, PH=2, PW=2, spatial_scale=1.0)
+    inp = si.roi_inputs(shape, 9, min_size=2.0)
+    inp["rois"][1, 0] = 5.0  # no such image
+    out = d.deform_roi_pool_forward(inp["x"].to(cuda_dev), inp["rois"].to(cuda_dev), inp["offset"].to(cuda_dev),
+                                    pooled=(2, 2), spatial_scale=1.0)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out[1]) == 0
+    keep = [0, 2]
+    ref = oracle.roi_pool_forward(inp["x"], inp["rois"][keep], inp["offset"][keep], pooled=(2, 2),
+                                  spatial_scale=1.0)
+    assert_close_fwd(out[keep], ref, "roi keep")
