@@ -192,6 +192,12 @@ __global__ void __launch_bounds__(kStagedMaxThreads, 1)
                     atomicOr(s.err, kDevErrTmaTimeout);
                     break;
                 }
+                // the second band of the CTA starts after the first has landed, so the
+                // first one is not slowed down by it at kernel start
+                if (n == 1 && nbuf == 2 && !mbar_wait_bounded(full_a, 0, kStagedWaitNs)) {
+                    atomicOr(s.err, kDevErrTmaTimeout);
+                    break;
+                }
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(full_a + 8 * b, (uint32_t)(sg.nbox * s.box_rows * s.row_bytes));
                 const uint32_t dst = smem_u32(smem + b * buf_bytes);
@@ -222,8 +228,8 @@ __global__ void __launch_bounds__(kStagedMaxThreads, 1)
         const long long it = sg.i0 + (long long)ch * IPW + ri;
         r_ok = sg.i0 < sg.i1 && it < sg.i1;
         if (!r_ok) return;
-        const long long plane = it / hw;
-        const int lp = (int)(it - plane * hw);
+        // pixel index inside the segment's (b, g) plane
+        const int lp = (int)(it - (long long)(sg.b * a.G + sg.g) * hw);
         r_ho = lp / a.Wo;
         r_wo = lp - r_ho * a.Wo;
         const long long mi = ((long long)sg.b * hw + lp) * a.G + sg.g;
@@ -272,41 +278,41 @@ __global__ void __launch_bounds__(kStagedMaxThreads, 1)
                     for (int j = 0; j < NT; ++j) m[j] *= inv;
                 }
                 unsigned fmask = 0;  // points of item ri read from global memory (this lane's share)
+                const float Hf = (float)a.H, Wf = (float)a.W;
 #pragma unroll
                 for (int j = 0; j < NT; ++j) {
                     const int k = k0 + j * L;
                     if (k >= K) continue;
-                    float4 w = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                    int2 ad = make_int2(0, 0);  // column 0 of the band: zeros
-                    if (r_ok) {
-                        const int2 kt = ktab[k];
-                        const float2 d = raw[j].pair();
-                        const float px = fmaf(a.offset_scale, d.x, (float)(r_wo * a.sw - a.pw + kt.y));
-                        const float py = fmaf(a.offset_scale, d.y, (float)(r_ho * a.sh - a.ph + kt.x));
-                        Tap tp{0, 0, 0.0f, 0.0f};
-                        const int st = make_tap(py, px, a.H, a.W, tp);
-                        if (st < 0) {
-                            const float nan = __int_as_float(0x7fc00000);
-                            w = make_float4(nan, nan, nan, nan);
-                        } else if (st > 0) {
-                            const float mk = m[j];
-                            const float tx0 = (1.0f - tp.lx) * mk, tx1 = tp.lx * mk;
-                            const float w00 = fmaf(-tx0, tp.ly, tx0), w10 = tx0 * tp.ly;
-                            const float w01 = fmaf(-tx1, tp.ly, tx1), w11 = tx1 * tp.ly;
-                            if (tp.y0 >= sg.ys && tp.y0 + 1 <= sg.ye) {
-                                const int P = ((tp.y0 - sg.ys) * W2 + tp.x0 + 1) * RB;
-                                const int order = (RB == 64) ? (((P >> 6) ^ ri) & 1) : 0;
-                                ad = order ? make_int2(P + RB, P) : make_int2(P, P + RB);
-                                w = order ? make_float4(w01, w11, w00, w10) : make_float4(w00, w10, w01, w11);
-                            } else {
-                                // inside the map, outside the staged rows: the staged pass reads
-                                // zeros here and the fallback pass adds the global corners
-                                w = make_float4(w00, w10, w01, w11);
-                                rec_f[k * IPW + ri] = (tp.y0 + 1) * W2 + tp.x0 + 1;
-                                fmask |= 1u << k;
-                            }
-                        }
-                    }
+                    // Branch-free: every lane of the warp takes the same instructions,
+                    // whatever case its tap falls in.
+                    const int2 kt = ktab[k];
+                    const float2 d = raw[j].pair();
+                    const float px = fmaf(a.offset_scale, d.x, (float)(r_wo * a.sw - a.pw + kt.y));
+                    const float py = fmaf(a.offset_scale, d.y, (float)(r_ho * a.sh - a.ph + kt.x));
+                    const float fy = floorf(py), fx = floorf(px);
+                    const float ly = py - fy, lx = px - fx;  // NaN for a NaN position
+                    const bool nanp = (px != px) | (py != py);
+                    // some neighbour inside the map (false for NaN and infinite positions)
+                    const bool inmap = (py > -1.0f) & (py < Hf) & (px > -1.0f) & (px < Wf);
+                    const int y0 = (int)fy, x0 = (int)fx;  // meaningful only when inmap
+                    const bool inband = (unsigned)y0 - (unsigned)sg.ys < (unsigned)(sg.ye - sg.ys);
+                    const bool smem_tap = r_ok & inmap & inband;
+                    const bool fb_tap = r_ok & inmap & !inband;
+                    const float mk = m[j];
+                    const float tx0 = (1.0f - lx) * mk, tx1 = lx * mk;
+                    const float w00 = fmaf(-tx0, ly, tx0), w10 = tx0 * ly;
+                    const float w01 = fmaf(-tx1, ly, tx1), w11 = tx1 * ly;
+                    const int P = (int)((((unsigned)y0 - (unsigned)sg.ys) * (unsigned)W2 + (unsigned)x0 + 1u) *
+                                        (unsigned)RB);
+                    const bool order = (RB == 64) && ((((unsigned)P >> 6) ^ (unsigned)ri) & 1u);
+                    int2 ad = order ? make_int2(P + RB, P) : make_int2(P, P + RB);
+                    if (!smem_tap) ad = make_int2(0, 0);  // column 0 of the band: zeros
+                    float4 w = (smem_tap && order) ? make_float4(w01, w11, w00, w10) : make_float4(w00, w10, w01, w11);
+                    if (!(r_ok & (inmap | nanp))) w = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    // inside the map, outside the staged rows: the staged pass reads zeros
+                    // here and the fallback pass adds the global corners
+                    if (fb_tap) rec_f[k * IPW + ri] = (y0 + 1) * W2 + x0 + 1;
+                    fmask |= (unsigned)fb_tap << k;
                     rec_w[k * IPW + ri] = w;
                     rec_a[k * IPW + ri] = ad;
                 }
@@ -335,16 +341,16 @@ __global__ void __launch_bounds__(kStagedMaxThreads, 1)
             float2 acc[V2];
 #pragma unroll
             for (int v = 0; v < V2; ++v) acc[v] = make_float2(0.0f, 0.0f);
-            const unsigned char *bq = band + q * 16;
+            const uint32_t bqa = smem_u32(band) + q * 16;  // 32-bit shared addresses
 #pragma unroll
             for (int k = 0; k < KMAX; ++k) {
                 if (k >= K) break;
                 const float4 w = rec_w[k * IPW + gi];
                 const int2 ad = rec_a[k * IPW + gi];
-                const uint4 va = *reinterpret_cast<const uint4 *>(bq + ad.x);
-                const uint4 vb = *reinterpret_cast<const uint4 *>(bq + ad.x + s.row_bytes);
-                const uint4 vc = *reinterpret_cast<const uint4 *>(bq + ad.y);
-                const uint4 vd = *reinterpret_cast<const uint4 *>(bq + ad.y + s.row_bytes);
+                const uint4 va = lds16(bqa + ad.x);
+                const uint4 vb = lds16(bqa + ad.x + s.row_bytes);
+                const uint4 vc = lds16(bqa + ad.y);
+                const uint4 vd = lds16(bqa + ad.y + s.row_bytes);
                 float2 f[V2];
                 unpack16x2<T>(va, f);
 #pragma unroll
