@@ -69,6 +69,8 @@ def _bind(lib):
     lib.oracle_agg_backward.restype = None
     lib.oracle_roi_pool_forward.argtypes = [i] * 8 + [ctypes.c_float, ctypes.c_float, dp, fp, fp, dp]
     lib.oracle_roi_pool_forward.restype = None
+    lib.oracle_pointwise_projection.argtypes = [ctypes.c_longlong, i, i, dp, dp, dp, dp]
+    lib.oracle_pointwise_projection.restype = None
     return lib
 
 
@@ -110,6 +112,27 @@ def dcn_forward(x, offset, mask, *, G: int, kh: int = 3, kw: int = 3, stride=(1,
                            _ptr(offset, ctypes.c_double), _ptr(mask, ctypes.c_double),
                            _ptr(out, ctypes.c_double))
     return out
+
+
+def pointwise_projection(v, weight, bias=None, *, lib=None) -> np.ndarray:
+    """out [..., Cout] = bias + v [..., Cin] . weight[Cout, Cin]^T in fp64 (1x1 convolution with bias)."""
+    lib = lib or load()
+    v, weight = _f64(v), _f64(weight)
+    Cout, Cin = weight.shape
+    assert v.shape[-1] == Cin, (v.shape, weight.shape)
+    npix = int(np.prod(v.shape[:-1]))
+    b = None if bias is None else _f64(bias)
+    assert b is None or b.shape == (Cout,)
+    out = np.empty(v.shape[:-1] + (Cout,), dtype=np.float64)
+    lib.oracle_pointwise_projection(npix, Cin, Cout, _ptr(v, ctypes.c_double), _ptr(weight, ctypes.c_double),
+                                    None if b is None else _ptr(b, ctypes.c_double), _ptr(out, ctypes.c_double))
+    return out
+
+
+def dcn_forward_proj(x, offset, mask, weight, bias=None, *, G: int, lib=None, **core) -> np.ndarray:
+    """The sampling core followed by its pointwise projection, both in fp64:
+    pointwise_projection(dcn_forward(x, offset, mask, ...), weight, bias)."""
+    return pointwise_projection(dcn_forward(x, offset, mask, G=G, lib=lib, **core), weight, bias, lib=lib)
 
 
 def dcn_backward(x, offset, mask, grad_out, *, G: int, kh: int = 3, kw: int = 3, stride=(1, 1),

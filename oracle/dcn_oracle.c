@@ -27,6 +27,9 @@
  *   Multi-camera multi-scale aggregation (Sparse4D deformable_aggregation
  *   article, sections 1, 2.1 and 2.2).
  *
+ *   The pointwise projection (1x1 convolution with bias) that follows the
+ *   core in the DCNv4 module (YOLOv11 + DCNv4 article, section 3.2).
+ *
  * Readings where the pages are silent (each one is listed in the design notes):
  *   - base grid point of kernel point (i,j) at output (ho,wo):
  *       y = ho*stride_h - pad_h + i*dil_h,  x = wo*stride_w - pad_w + j*dil_w,
@@ -148,6 +151,30 @@ void oracle_dcn_forward(int B, int H, int W, int G, int C, int kh, int kw,
                 }
             free(m);
         }
+}
+
+/*
+ * Pointwise projection after the sampling core (the 1x1 convolution with bias
+ * that the DCNv4 module of the YOLOv11 + DCNv4 article, section 3.2, applies
+ * to the core's output):
+ *     out[p, o] = bias[o] + sum_c Wt[o, c] * in[p, c]
+ * for every pixel p of the NHWC map; Wt is [Cout, Cin] (a Conv2d weight with
+ * its 1x1 spatial extent dropped); bias may be NULL (no bias).
+ */
+void oracle_pointwise_projection(long long npix, int Cin, int Cout, const double *in, const double *Wt,
+                                 const double *bias, double *out)
+{
+#pragma omp parallel for schedule(static)
+    for (long long p = 0; p < npix; ++p) {
+        const double *v = in + (size_t)p * Cin;
+        double *y = out + (size_t)p * Cout;
+        for (int o = 0; o < Cout; ++o) {
+            const double *w = Wt + (size_t)o * Cin;
+            double s = bias ? bias[o] : 0.0;
+            for (int c = 0; c < Cin; ++c) s += w[c] * v[c];
+            y[o] = s;
+        }
+    }
 }
 
 /*

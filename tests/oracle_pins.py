@@ -547,3 +547,52 @@ def pin_roi_torchvision(lib):
 
 ROI_PINS = [pin_roi_brute_force, pin_roi_affine, pin_roi_constant, pin_roi_torchvision]
 ALL_PINS = ALL_PINS + ROI_PINS
+
+
+# ---------------------------------------------------------------- pointwise projection pins
+def pin_proj_conv2d(lib):
+    """The projection equals PyTorch's 1x1 convolution with bias (fp64), Cout != Cin."""
+    rng = np.random.default_rng(101)
+    v = rng.standard_normal((2, 5, 7, 12))
+    w = rng.standard_normal((20, 12))
+    b = rng.standard_normal(20)
+    out = oracle.pointwise_projection(v, w, b, lib=lib)
+    ref = torch.nn.functional.conv2d(torch.from_numpy(v).permute(0, 3, 1, 2), torch.from_numpy(w)[:, :, None, None],
+                                     torch.from_numpy(b))
+    assert np.allclose(out, ref.permute(0, 2, 3, 1).numpy(), rtol=0, atol=1e-12), "projection vs conv2d"
+    out0 = oracle.pointwise_projection(v, w, None, lib=lib)
+    ref0 = torch.nn.functional.conv2d(torch.from_numpy(v).permute(0, 3, 1, 2), torch.from_numpy(w)[:, :, None, None])
+    assert np.allclose(out0, ref0.permute(0, 2, 3, 1).numpy(), rtol=0, atol=1e-12), "projection without bias"
+
+
+def pin_proj_closed_forms(lib):
+    """A permutation matrix permutes channels exactly; a zero matrix leaves the bias."""
+    rng = np.random.default_rng(102)
+    v = rng.standard_normal((3, 4, 16))
+    perm = rng.permutation(16)
+    w = np.eye(16)[perm]  # out[o] = v[perm[o]]
+    assert np.array_equal(oracle.pointwise_projection(v, w, lib=lib), v[..., perm]), "projection permutation"
+    b = rng.standard_normal(9)
+    out = oracle.pointwise_projection(v, np.zeros((9, 16)), b, lib=lib)
+    assert np.array_equal(out, np.broadcast_to(b, out.shape)), "projection bias only"
+
+
+def pin_proj_composed_identity(lib):
+    """Zero offsets with a one-hot centre mask make the core the identity (3x3, pad 1), so the
+    composed operator is a 1x1 convolution of x itself."""
+    rng = np.random.default_rng(103)
+    B, H, W, G, C = 2, 6, 5, 2, 8
+    x = rng.standard_normal((B, H, W, G * C))
+    off = np.zeros((B, H, W, G, 9, 2))
+    mask = np.zeros((B, H, W, G, 9))
+    mask[..., 4] = 1.0
+    w = rng.standard_normal((24, G * C))
+    b = rng.standard_normal(24)
+    out = oracle.dcn_forward_proj(x, off, mask, w, b, G=G, lib=lib)
+    ref = torch.nn.functional.conv2d(torch.from_numpy(x).permute(0, 3, 1, 2), torch.from_numpy(w)[:, :, None, None],
+                                     torch.from_numpy(b))
+    assert np.allclose(out, ref.permute(0, 2, 3, 1).numpy(), rtol=0, atol=1e-12), "composed identity"
+
+
+PROJ_PINS = [pin_proj_conv2d, pin_proj_closed_forms, pin_proj_composed_identity]
+ALL_PINS = ALL_PINS + PROJ_PINS

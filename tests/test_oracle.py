@@ -106,6 +106,14 @@ MUTATIONS = [
      pins.ROI_PINS),
     ("const float x1 = r[1] * spatial_scale, y1 = r[2] * spatial_scale;",
      "const float x1 = r[1], y1 = r[2] * spatial_scale;", 0, pins.ROI_PINS),
+    ("const double *w = Wt + (size_t)o * Cin;", "const double *w = Wt + (size_t)o;", 0, pins.PROJ_PINS),
+    # weight read as [Cin, Cout] (transposed; every index stays inside the array)
+    ("const double *w = Wt + (size_t)o * Cin;\n            double s = bias ? bias[o] : 0.0;\n"
+     "            for (int c = 0; c < Cin; ++c) s += w[c] * v[c];",
+     "const double *w = Wt + (size_t)o;\n            double s = bias ? bias[o] : 0.0;\n"
+     "            for (int c = 0; c < Cin; ++c) s += w[(size_t)c * Cout] * v[c];", 0, pins.PROJ_PINS),
+    ("double s = bias ? bias[o] : 0.0;", "double s = 0.0;", 0, pins.PROJ_PINS),
+    ("double s = bias ? bias[o] : 0.0;", "double s = bias ? bias[0] : 0.0;", 0, pins.PROJ_PINS),
 ]
 
 
