@@ -16,7 +16,9 @@
 // 16-byte vector reductions.
 //
 // Taken when G*C*sizeof(T) is 512, 1024 or 2048 bytes; other widths use the
-// per-group kernels in deform_agg.cu.
+// per-group kernels in deform_agg.cu.  For fp32 outputs the forward uses
+// pair-granular persistent warps (agg_forward_pairs_f32) instead of one CTA
+// per anchor, for load balance.
 #include "dcn_atomic.cuh"
 #include "dcn_launch.h"
 
@@ -118,6 +120,120 @@ __global__ void __launch_bounds__(kAggWarps * 32) agg_forward_wide(AggArgs a) {
             f[v] = nan_any ? __int_as_float(0x7fc00000) : sum;
         }
         *reinterpret_cast<uint4 *>(out + c * V) = pack16<T>(f);
+    }
+}
+
+// fp32 variant with pair-granular persistent work: warp w of the grid owns the
+// contiguous range of (anchor, pair) units [U*w/NW, U*(w+1)/NW), so every warp
+// gets the same number of samples whatever the anchor count.  Consecutive
+// units of one anchor accumulate in registers; when the anchor changes the
+// partial row is added to the (zeroed) output with 16-byte reductions, so an
+// anchor split between two warps is summed in L2 (a few flushes per warp).
+// The next unit's location is loaded one unit ahead, and the four corner
+// loads of a sample are issued unconditionally (an out-of-map corner loads
+// nothing and gets weight zero), so the unrolled scale loop keeps several
+// samples' loads in flight.
+template <int CPL>
+__global__ void __launch_bounds__(kAggWarps * 32) agg_forward_pairs_f32(AggArgs a, long long units, int total_warps) {
+    constexpr int V = 4;
+    constexpr int ROW = CPL * 32 * V;
+    __shared__ int4 tab[kAggTableMax];
+    const int lane = threadIdx.x & 31;
+    const int CS = a.cams * a.scales;
+    const bool tab_smem = CS <= kAggTableMax;
+    if (tab_smem)
+        for (int i = threadIdx.x; i < CS; i += blockDim.x) tab[i] = load_table(a, i);
+    __syncthreads();
+
+    const int gw = blockIdx.x * kAggWarps + (threadIdx.x >> 5);
+    const long long u0 = units * gw / total_warps, u1 = units * (gw + 1) / total_warps;
+    if (u0 >= u1) return;
+    const int pairs = a.P * a.cams;
+    const float *__restrict__ wts = static_cast<const float *>(a.weights);
+    float *__restrict__ out = static_cast<float *>(a.out);
+    int grp[CPL];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) grp[j] = (32 * j + lane) * V / a.C;
+    float acc[CPL][V];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j)
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[j][v] = 0.0f;
+    bool nan_pos = false;
+
+    const float2 *locp = reinterpret_cast<const float2 *>(a.loc);
+    float2 uv_next = __ldg(locp + u0);  // unit index == (b*A + anchor)*pairs + pair
+    long long ba = u0 / pairs;
+    for (long long u = u0; u < u1; ++u) {
+        const float2 uv = uv_next;
+        if (u + 1 < u1) uv_next = __ldg(locp + u + 1);
+        const long long bau = u / pairs;
+        if (bau != ba) {  // flush the finished anchor
+            float *o = out + ba * ROW + lane * V;
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                if (nan_pos) {
+#pragma unroll
+                    for (int v = 0; v < V; ++v) acc[j][v] = __int_as_float(0x7fc00000);
+                }
+                red_add16<float>(o + 32 * j * V, acc[j]);
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[j][v] = 0.0f;
+            }
+            nan_pos = false;
+            ba = bau;
+        }
+        const int pc = (int)(u - bau * pairs);
+        const int cam = pc % a.cams;
+        const int b = (int)(bau / a.A);
+        const float *feat = static_cast<const float *>(a.feat) + (long long)b * a.rows * ROW;
+        const long long wbase = u * a.scales;
+#pragma unroll 4
+        for (int s = 0; s < a.scales; ++s) {
+            const int4 t = tab_smem ? tab[cam * a.scales + s] : load_table(a, cam * a.scales + s);
+            const float px = fmaf(uv.x, (float)t.y, -0.5f);
+            const float py = fmaf(uv.y, (float)t.x, -0.5f);
+            Tap tp{0, 0, 0.0f, 0.0f};
+            const int st = make_tap(py, px, t.x, t.y, tp);
+            nan_pos |= st < 0;
+            float w[CPL];
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) w[j] = __ldg(wts + (wbase + s) * a.G + grp[j]);
+            float g[4];
+            float4 f[4][CPL];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int y = tp.y0 + (c >> 1), x = tp.x0 + (c & 1);
+                const long long row = (long long)t.z + (long long)y * t.y + x;
+                const bool ok = st > 0 && y >= 0 && y < t.x && x >= 0 && x < t.y && row >= 0 && row < a.rows;
+                g[c] = ok ? ((c >> 1) ? tp.ly : 1.0f - tp.ly) * ((c & 1) ? tp.lx : 1.0f - tp.lx) : 0.0f;
+                const float *r = feat + (ok ? row : 0) * ROW + lane * V;
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) {
+                    f[c][j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    if (ok) f[c][j] = __ldg(reinterpret_cast<const float4 *>(r + 32 * j * V));
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) {
+                    const float wg = w[j] * g[c];
+                    acc[j][0] = fmaf(wg, f[c][j].x, acc[j][0]);
+                    acc[j][1] = fmaf(wg, f[c][j].y, acc[j][1]);
+                    acc[j][2] = fmaf(wg, f[c][j].z, acc[j][2]);
+                    acc[j][3] = fmaf(wg, f[c][j].w, acc[j][3]);
+                }
+        }
+    }
+    float *o = out + ba * ROW + lane * V;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        if (nan_pos) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[j][v] = __int_as_float(0x7fc00000);
+        }
+        red_add16<float>(o + 32 * j * V, acc[j]);
     }
 }
 
@@ -238,6 +354,19 @@ cudaError_t launch(const AggArgs &a, bool bwd, cudaStream_t stream) {
         cudaError_t e = cudaMemsetAsync(a.grad_feat, 0, (size_t)a.B * a.rows * a.G * a.C * sizeof(T), stream);
         if (e != cudaSuccess) return e;
         agg_backward_wide<T, CPL><<<grid, kAggWarps * 32, 0, stream>>>(a);
+    } else if (sizeof(T) == 4) {
+        // fp32 output: pair-granular persistent warps, partial rows added in L2
+        int dev = 0, sms = 148, per_sm = 1;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, agg_forward_pairs_f32<CPL>, kAggWarps * 32, 0);
+        if (per_sm < 1) per_sm = 1;
+        const long long units = (long long)a.B * a.A * a.P * a.cams;
+        long long ctas = (long long)sms * per_sm;
+        if (ctas * kAggWarps > units) ctas = (units + kAggWarps - 1) / kAggWarps;
+        cudaError_t e = cudaMemsetAsync(a.out, 0, (size_t)a.B * a.A * a.G * a.C * sizeof(float), stream);
+        if (e != cudaSuccess) return e;
+        agg_forward_pairs_f32<CPL><<<(unsigned)ctas, kAggWarps * 32, 0, stream>>>(a, units, (int)(ctas * kAggWarps));
     } else {
         agg_forward_wide<T, CPL><<<grid, kAggWarps * 32, 0, stream>>>(a);
     }
