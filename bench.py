@@ -41,8 +41,11 @@ WORKLOAD = ("DCNv4 core forward, YOLO-P4 shape: B=8 per GPU, H=W=40, 512 ch as G
             "offsets~N(0,3), mask~N(0,1)")
 FALLBACK_HBM_GBS = 6650.0
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+# Sources of the timed forward kernel: the recorded DRAM traffic is used only
+# while these are unchanged.
 KERNEL_SOURCES = [os.path.join(ROOT, "deformable_convolution_sampling_dcn_b200", "csrc", f)
-                  for f in ("dcn_forward_plane.cu", "dcn_forward_generic.cu", "dcn_common.cuh")]
+                  for f in ("dcn_forward_plane.cu", "dcn_forward_staged.cuh", "dcn_forward_staged_f16.cu",
+                            "dcn_tma.cuh", "dcn_forward_generic.cu", "dcn_common.cuh")]
 
 
 def kernel_hash() -> str:
@@ -417,6 +420,37 @@ def measure_rows(dcn, dev, stream, l2, barrier, world, steps=280):
     ms = time_steps(mkr, sets, steps, 3 * R, stream, barrier, world) / steps
     out["roi_pool"] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(rs.samples / ms / 1e6, 2),
                        "GB_s": round(rs.compulsory_bytes() / ms / 1e6, 1), "R": R}
+    del sets
+
+    # DCNv4 P4 core fused with its 512 -> 512 projection (tensor cores), and for
+    # context the same two steps unfused: the core kernel, then a cuBLAS GEMM
+    # through torch on the stored core output.
+    shape, inp = si.workload_proj()
+    t = [inp[k].to(dev) for k in ("x", "offset", "mask", "weight", "bias")]
+    cout = t[3].shape[0]
+    pbytes = shape.compulsory_bytes() + (t[3].numel() + t[4].numel()) * 2 + \
+        shape.B * shape.Ho * shape.Wo * (cout - shape.G * shape.C) * 2
+    R = max(2, math.ceil(4 * l2 / pbytes))
+    sets = [[u.clone() for u in t] + [torch.empty((shape.B, shape.Ho, shape.Wo, cout), dtype=t[0].dtype, device=dev),
+                                      torch.empty((shape.B, shape.Ho, shape.Wo, shape.G * shape.C),
+                                                  dtype=t[0].dtype, device=dev)] for _ in range(R)]
+
+    def mkp(s):
+        return lambda: dcn.dcn_core_forward_proj(s[0], s[1], s[2], s[3], s[4], group=shape.G, out=s[5])
+
+    ms = time_steps(mkp, sets, steps, 3 * R, stream, barrier, world) / steps
+
+    def mku(s):
+        def call():
+            dcn.dcn_core_forward(s[0], s[1], s[2], group=shape.G, out=s[6])
+            torch.addmm(s[4], s[6].view(-1, shape.G * shape.C), s[3].t(), out=s[5].view(-1, cout))
+        return call
+
+    ms_u = time_steps(mku, sets, steps, 3 * R, stream, barrier, world) / steps
+    flops = 2.0 * shape.B * shape.Ho * shape.Wo * cout * shape.G * shape.C
+    out["dcnv4_p4_proj"] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(shape.samples / ms / 1e6, 2),
+                            "GB_s": round(pbytes / ms / 1e6, 1), "gemm_TFLOP_s": round(flops / ms / 1e9, 1),
+                            "unfused_core_then_cublas_us": round(ms_u * 1e3, 2), "Cout": cout, "R": R}
     return out
 
 

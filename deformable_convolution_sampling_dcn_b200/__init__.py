@@ -3,6 +3,7 @@
 Thin Python front end of libdcn_b200.so (C ABI in include/dcn_b200.h):
 
     dcn_core_forward / dcn_core_backward     DCNv2/v3/v4 sampling core
+    dcn_core_forward_proj                    the core fused with its 1x1 projection (DCNv4 module)
     deform_agg_forward / deform_agg_backward Sparse4D multi-camera aggregation
     deform_roi_pool_forward                  deformable RoI pooling
     DCNCoreFunction, DeformAggFunction       autograd wrappers over the above
@@ -18,10 +19,11 @@ from typing import Tuple
 import torch
 
 from ._binding import (ABI_VERSION, EXPORTS, DaggParams, DcnError, DcnParams, DroiParams, core_params,
-                       dcn_core_backward, dcn_core_forward, dcn_core_output_hw, deform_agg_backward,
+                       dcn_core_backward, dcn_core_forward, dcn_core_forward_proj, dcn_core_output_hw,
+                       deform_agg_backward,
                        deform_agg_forward, deform_roi_pool_forward, lib)
 
-__all__ = ["dcn_core_forward", "dcn_core_backward", "dcn_core_output_hw", "deform_agg_forward",
+__all__ = ["dcn_core_forward", "dcn_core_forward_proj", "dcn_core_backward", "dcn_core_output_hw", "deform_agg_forward",
            "deform_agg_backward", "deform_roi_pool_forward", "DroiParams", "DCNCoreFunction", "DeformAggFunction", "shard_range", "lib", "DcnError",
            "DcnParams", "DaggParams", "core_params", "EXPORTS", "ABI_VERSION"]
 

@@ -156,6 +156,38 @@ dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offs
     return cuda_status(e, "dcn_core_forward launch");
 }
 
+dcn_status dcn_core_forward_proj(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
+                                 const void *mask, const void *weight, const void *bias, void *out,
+                                 dcn_stream_t stream) {
+    int Ho, Wo;
+    dcn_status s = check_core(p, &Ho, &Wo);
+    if (s != DCN_OK) return s;
+    if (p->dtype != DCN_F16 && p->dtype != DCN_BF16)
+        return fail(DCN_ERR_UNSUPPORTED, "the fused projection takes fp16 or bf16 (dtype %d)", p->dtype);
+    if (p->C > 64) return fail(DCN_ERR_UNSUPPORTED, "the fused projection takes C <= 64 (C = %d)", p->C);
+    const long long GC = (long long)p->G * p->C;
+    if (GC % 64 != 0 || GC > 512)
+        return fail(DCN_ERR_UNSUPPORTED, "the fused projection takes G*C in {64, 128, ..., 512} (G*C = %lld)", GC);
+    if ((long long)p->kh * p->kw > 25)
+        return fail(DCN_ERR_UNSUPPORTED, "the fused projection takes kh*kw <= 25");
+    if (Cout < 8 || Cout > 512 || Cout % 8 != 0)
+        return fail(DCN_ERR_UNSUPPORTED, "Cout must be a multiple of 8 in [8, 512] (Cout = %d)", Cout);
+    if (p->B == 0) return DCN_OK;
+    if (!x || !offset || !mask || !weight || !out)
+        return fail(DCN_ERR_NULL, "x, offset, mask, weight and out are required");
+    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(weight, 16))
+        return fail(DCN_ERR_ALIGN, "x, weight and out must be 16-byte aligned");
+    if (!aligned(offset, 4) || !aligned(mask, 2) || !aligned(bias, 2))
+        return fail(DCN_ERR_ALIGN, "offset must be 4-byte aligned, mask and bias 2-byte aligned");
+    dcnb::ProjArgs a;
+    a.core = core_args(p, Ho, Wo);
+    a.core.x = x; a.core.offset = offset; a.core.mask = mask; a.core.out = out;
+    a.weight = weight;
+    a.bias = bias;
+    a.Cout = Cout;
+    return cuda_status(dcnb::launch_core_forward_proj(a, (cudaStream_t)stream), "dcn_core_forward_proj launch");
+}
+
 dcn_status dcn_core_backward(const dcn_params *p, const void *x, const void *offset, const void *mask,
                              const void *grad_out, void *grad_x, void *grad_offset, void *grad_mask,
                              dcn_stream_t stream) {

@@ -8,6 +8,7 @@
 
 #include <mutex>
 
+#include "dcn_device.h"
 #include "dcn_forward_staged.cuh"
 
 namespace dcnb {
@@ -22,11 +23,6 @@ cudaError_t take_device_error(unsigned int *value) {
     return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
 }
 
-namespace {
-
-constexpr int kHaloMax = 8;   // rows of margin for the offsets
-constexpr int kBoxRows = 4;   // rows per TMA box
-
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -40,13 +36,6 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-struct DeviceInfo {
-    int sms = 0, smem_optin = 0, smem_per_sm = 0;
-    unsigned int *err = nullptr;
-};
-
-// Per-device facts, looked up once per device (the error word's address is
-// per device context).
 const DeviceInfo *device_info() {
     constexpr int kMaxDev = 64;
     static DeviceInfo info[kMaxDev];
@@ -63,6 +52,11 @@ const DeviceInfo *device_info() {
     });
     return info[dev].err ? &info[dev] : nullptr;
 }
+
+namespace {
+
+constexpr int kHaloMax = 8;   // rows of margin for the offsets
+constexpr int kBoxRows = 4;   // rows per TMA box
 
 template <typename T>
 cudaError_t launch_t(const CoreArgs &a, cudaStream_t stream, bool *handled) {

@@ -27,6 +27,14 @@ struct CoreArgs {
     DType dtype;
 };
 
+// Forward core followed by its pointwise projection (fp16/bf16 only).
+struct ProjArgs {
+    CoreArgs core;       // core.out is the projected output [B, Ho, Wo, Cout]
+    const void *weight;  // [Cout, G*C]
+    const void *bias;    // [Cout] or nullptr
+    int Cout;
+};
+
 struct AggArgs {
     const void *feat;
     const int32_t *spatial_shape;
@@ -62,6 +70,8 @@ cudaError_t launch_core_forward_plane(const CoreArgs &a, cudaStream_t stream, bo
 // Reads and clears the device error word that bounded waits set (bit 0:
 // a TMA wait ran out).  Synchronous.
 cudaError_t take_device_error(unsigned int *value);
+// Fused core + projection (tcgen05 GEMM on the core tile in shared memory).
+cudaError_t launch_core_forward_proj(const ProjArgs &a, cudaStream_t stream);
 cudaError_t launch_agg_forward(const AggArgs &a, cudaStream_t stream);
 // Anchor-wide aggregation kernels (all groups per CTA); sets *handled = false
 // (and launches nothing) when the feature row width does not fit them.

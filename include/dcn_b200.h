@@ -13,8 +13,9 @@
  * sum_n m(pn) w(pn) x(p + pn + dpn)), either normalised by a softmax over the K
  * points of the (pixel, group) as in DCNv3 or used raw as in DCNv4 (YOLOv11 +
  * DCNv4 article, section 1.1), and the K samples are summed in fp32.  The
- * dense weight w(pn) of DCNv1/v2 is not part of this library: it is a plain
- * convolution the caller runs before or after.
+ * pointwise projection that follows the core in the DCNv4 module (1x1
+ * convolution with bias) is available fused with it (dcn_core_forward_proj);
+ * the dense per-point weight w(pn) of DCNv1/v2 is not part of this library.
  *
  * Conventions shared by every call:
  *   - All tensor pointers are DEVICE pointers to dense, C-contiguous buffers
@@ -97,13 +98,37 @@ dcn_status dcn_core_output_hw(const dcn_params *p, int32_t *Ho, int32_t *Wo);
  * Forward core: out = sum_k m_k * bilinear(x, p_k) per (pixel, group).
  * Reads x, offset, mask; overwrites every element of out.
  * Two kernels implement it: a shared-memory staged one (group rows of 32 to
- * 256 bytes, W <= 254, K <= 64) and a generic one for every other shape.
+ * 256 bytes, W <= 254, K <= 25) and a generic one for every other shape.
  * Setting the environment variable DCN_B200_FORCE_GENERIC=1 routes every
  * call to the generic kernel (both give the same result up to fp32
  * summation order).
  */
 dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offset,
                             const void *mask, void *out, dcn_stream_t stream);
+
+/*
+ * Forward core followed by its pointwise projection, in one kernel (the
+ * DCNv4 module of the YOLOv11 + DCNv4 article, section 3.2, passes the core's
+ * output through a 1x1 convolution with bias):
+ *   out[b, ho, wo, o] = bias[o] + sum_j weight[o, j] * core[b, ho, wo, j],
+ *   j = g*C + c over the G*C core channels.
+ *   weight [Cout, G*C]        storage dtype (a Conv2d weight without its 1x1 extent)
+ *   bias   [Cout]             storage dtype, or NULL for no bias
+ *   out    [B, Ho, Wo, Cout]  storage dtype
+ * x, offset and mask are as for dcn_core_forward.  The core value of each
+ * (pixel, channel) is accumulated in fp32 and rounded once to the storage
+ * dtype (what dcn_core_forward would store); the projection runs on the
+ * tensor cores with fp32 accumulation, adds the bias in fp32 and rounds the
+ * result once.  The core never reaches device memory.
+ * Supported: fp16 and bf16 (fp32 returns DCN_ERR_UNSUPPORTED), C <= 64 with
+ * G*C a multiple of 64 up to 512, kh*kw <= 25, Cout a multiple of 8 in
+ * [8, 512]; both mask modes.  x, weight and out 16-byte aligned, offset
+ * 4-byte, mask and bias 2-byte.  A NaN sampling position makes every output
+ * channel of its pixel NaN.
+ */
+dcn_status dcn_core_forward_proj(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
+                                 const void *mask, const void *weight, const void *bias, void *out,
+                                 dcn_stream_t stream);
 
 /*
  * Backward core: gradients of L = <grad_out, out> with respect to x, offset

@@ -298,3 +298,25 @@ def roi_inputs(shape: RoiShape, seed: int, *, offset_std: float = 1.0,
     off = rng.standard_normal((s.N, s.PH, s.PW, 2)) * offset_std
     return {"x": _round(x, s.dtype), "rois": torch.from_numpy(rois),
             "offset": torch.from_numpy(off.astype(np.float32))}
+
+
+# The DCNv4 module's pointwise projection after the core (a 1x1 convolution
+# with bias, channels -> channels): at the P4 shape, G*C = 512 -> 512.
+PROJ_COUT_P4 = 512
+SEEDS["dcnv4_p4_proj"] = 6
+
+
+def proj_inputs(cin: int, cout: int, dtype: str, seed: int) -> Dict[str, torch.Tensor]:
+    """weight [cout, cin] ~ N(0, 1/cin) (unit-variance outputs for unit-variance
+    inputs) and bias [cout] ~ N(0, 0.1^2), rounded once to the storage dtype."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    w = rng.standard_normal((cout, cin)) / np.sqrt(cin)
+    b = rng.standard_normal(cout) * 0.1
+    return {"weight": _round(w, dtype), "bias": _round(b, dtype)}
+
+
+def workload_proj() -> Tuple[CoreShape, Dict[str, torch.Tensor]]:
+    """DCNv4 P4 core inputs plus its 512 -> 512 projection."""
+    shape, inp = workload_core("dcnv4_p4")
+    inp.update(proj_inputs(shape.G * shape.C, PROJ_COUT_P4, shape.dtype, SEEDS["dcnv4_p4_proj"]))
+    return shape, inp
