@@ -44,7 +44,7 @@ constexpr int kProjThreads = (kGatherWarps + 2) * 32;
 constexpr int kWStages = 4;
 constexpr int kWTileBytes = 128 * 128;  // 128 rows x 64 elements x 2 bytes
 constexpr int kMaxChunk = 128;          // pixels per chunk (MMA N <= 128)
-constexpr int kMaxKBlocks = 8;          // G*C <= 512
+constexpr int kBSlots = 4;             // B-operand ring: K-blocks in flight
 constexpr uint64_t kProjWaitNs = 1000000000ull;
 
 struct ProjParams {
@@ -149,34 +149,244 @@ __device__ __forceinline__ void chunk_range(long long r0, long long r1, int c, i
     c1 = r0 + len * (c + 1) / n;
 }
 
-template <typename T, int LPI, bool SOFTMAX, int KMAX>
+// Zeros read by the corners of a tap that lie outside the map (one group row
+// of at most 128 bytes).
+__device__ __align__(16) unsigned char g_zero_row[128];
+
+// Sampling of one 64-channel K-block of a chunk into its B-operand slot.
+//
+// RECORDS (K <= 9, 2..8 lanes per item): per warp step of IPW items, the
+// lanes first turn every (item, point) into a record in shared memory - the
+// four bilinear weights with the modulation folded in and the four corner
+// pixel indices (-1: outside the map, read from the zero row) - computed
+// once by one lane; then the LPI lanes of each item read the records and
+// gather their 16-byte channel chunks of the four corners through L1.
+// Otherwise every lane of an item computes the taps itself.
+// Items are enumerated group-major (pixels fastest), so consecutive items
+// of a warp sample neighbouring pixels of one group.
+template <typename T, int LPI, bool SOFTMAX, int KMAX, bool RECORDS>
+__device__ __forceinline__ void gather_kblock(const ProjParams &p, int kb, long long c0, int n_px, int warp,
+                                              int lane, unsigned char *slot, float4 *rec_w, int4 *rec_o,
+                                              const int2 *ktab) {
+    constexpr int V = Storage<T>::kVec;
+    constexpr int IPW = 32 / LPI;
+    constexpr int NT = (KMAX + LPI - 1) / LPI;  // records per lane and step
+    const CoreArgs &a = p.a;
+    const int K = a.kh * a.kw;
+    const int GC = a.G * a.C;
+    const int gpb = 64 / a.C;  // groups per K-block
+    const unsigned HoWo = (unsigned)a.Ho * (unsigned)a.Wo;
+    const T *__restrict__ xg = static_cast<const T *>(a.x);
+    const T *__restrict__ off = static_cast<const T *>(a.offset);
+    const T *__restrict__ msk = static_cast<const T *>(a.mask);
+    const int items = n_px * gpb;
+    const int gi = lane / LPI, q = lane % LPI;  // gather role
+    for (int base = warp * IPW; base < items; base += kGatherWarps * IPW) {
+        // the gather role's item
+        const int item = base + gi;
+        const bool valid = item < items;
+        const int gl = item / n_px, px = item - (item / n_px) * n_px;
+        const int g = kb * gpb + gl;
+        const unsigned pix = (unsigned)(c0 + px);
+        const unsigned b = pix / HoWo;
+        const T *xb = xg + (long long)b * a.H * a.W * GC + g * a.C + q * V;
+        float acc[V];
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = 0.0f;
+        if (RECORDS) {
+            // ---- records: lane (ri, k0) builds points k0, k0 + LPI, ... of item ri
+            const int ri = lane % IPW, k0 = lane / IPW;
+            const int item_r = base + ri;
+            const bool valid_r = item_r < items;
+            const int gl_r = item_r / n_px, px_r = item_r - (item_r / n_px) * n_px;
+            const unsigned pix_r = (unsigned)(c0 + px_r);
+            const unsigned rem = pix_r % HoWo;
+            const int ho = (int)(rem / (unsigned)a.Wo), wo = (int)(rem % (unsigned)a.Wo);
+            const long long mi = (long long)pix_r * a.G + kb * gpb + gl_r;
+            float dx[NT], dy[NT], m[NT];
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const int k = k0 + j * LPI;
+                dx[j] = dy[j] = 0.0f;
+                m[j] = SOFTMAX ? -INFINITY : 0.0f;
+                if (valid_r && k < K) {
+                    const float2 d = load_pair(off + (mi * K + k) * 2);
+                    dx[j] = d.x;
+                    dy[j] = d.y;
+                    m[j] = load_scalar(msk + mi * K + k);
+                }
+            }
+            if (SOFTMAX) {
+                float mx = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) mx = fmaxf(mx, m[j]);
+#pragma unroll
+                for (int o = IPW; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                float sum = 0.0f;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    m[j] = (k0 + j * LPI < K && valid_r) ? expf(m[j] - mx) : 0.0f;
+                    sum += m[j];
+                }
+#pragma unroll
+                for (int o = IPW; o < 32; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+                const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) m[j] *= inv;
+            }
+            const float Hf = (float)a.H, Wf = (float)a.W;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                const int k = k0 + j * LPI;
+                if (k >= K) continue;
+                const int2 kt = ktab[k];
+                const float pxf = fmaf(a.offset_scale, dx[j], (float)(wo * a.sw - a.pw + kt.y));
+                const float pyf = fmaf(a.offset_scale, dy[j], (float)(ho * a.sh - a.ph + kt.x));
+                const float fy = floorf(pyf), fx = floorf(pxf);
+                const float ly = pyf - fy, lx = pxf - fx;  // NaN for a NaN position
+                const bool nanp = (pxf != pxf) | (pyf != pyf);
+                const bool inmap = (pyf > -1.0f) & (pyf < Hf) & (pxf > -1.0f) & (pxf < Wf);
+                const int y0 = inmap ? (int)fy : -2, x0 = inmap ? (int)fx : -2;
+                const bool vy0 = (unsigned)y0 < (unsigned)a.H, vy1 = (unsigned)(y0 + 1) < (unsigned)a.H;
+                const bool vx0 = (unsigned)x0 < (unsigned)a.W, vx1 = (unsigned)(x0 + 1) < (unsigned)a.W;
+                const int r00 = y0 * a.W + x0;
+                int4 o4 = make_int4(vy0 & vx0 ? r00 : -1, vy0 & vx1 ? r00 + 1 : -1, vy1 & vx0 ? r00 + a.W : -1,
+                                    vy1 & vx1 ? r00 + a.W + 1 : -1);
+                const float mk = m[j];
+                const float tx0 = (1.0f - lx) * mk, tx1 = lx * mk;
+                float4 w4 = make_float4(fmaf(-tx0, ly, tx0), fmaf(-tx1, ly, tx1), tx0 * ly, tx1 * ly);
+                if (!(valid_r & (inmap | nanp))) w4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (!valid_r) o4 = make_int4(-1, -1, -1, -1);
+                rec_w[k * IPW + ri] = w4;  // a NaN position keeps NaN weights and zero-row corners
+                rec_o[k * IPW + ri] = o4;
+            }
+            __syncwarp();
+            // ---- gather
+            const unsigned char *zrow = g_zero_row + q * 16;
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k) {
+                if (k >= K) break;
+                const float4 w = rec_w[k * IPW + gi];
+                const int4 o = rec_o[k * IPW + gi];
+                const uint4 v0 = ld_nc16(o.x >= 0 ? (const void *)(xb + (long long)o.x * GC) : (const void *)zrow);
+                const uint4 v1 = ld_nc16(o.y >= 0 ? (const void *)(xb + (long long)o.y * GC) : (const void *)zrow);
+                const uint4 v2 = ld_nc16(o.z >= 0 ? (const void *)(xb + (long long)o.z * GC) : (const void *)zrow);
+                const uint4 v3 = ld_nc16(o.w >= 0 ? (const void *)(xb + (long long)o.w * GC) : (const void *)zrow);
+                float f[V];
+                unpack16<T>(v0, f);
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[v] = fmaf(w.x, f[v], acc[v]);
+                unpack16<T>(v1, f);
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[v] = fmaf(w.y, f[v], acc[v]);
+                unpack16<T>(v2, f);
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[v] = fmaf(w.z, f[v], acc[v]);
+                unpack16<T>(v3, f);
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[v] = fmaf(w.w, f[v], acc[v]);
+            }
+        } else if (valid) {
+            // ---- every lane computes the taps of its item
+            const unsigned rem = pix % HoWo;
+            const int ho = (int)(rem / (unsigned)a.Wo), wo = (int)(rem % (unsigned)a.Wo);
+            const long long mi = (long long)pix * a.G + g;
+            const T *o_item = off + mi * K * 2;
+            const T *m_item = msk + mi * K;
+            float mx = 0.0f, inv_sum = 1.0f;
+            if (SOFTMAX) {
+                mx = -INFINITY;
+                for (int k = 0; k < K; ++k) mx = fmaxf(mx, load_scalar(m_item + k));
+                float sum = 0.0f;
+                for (int k = 0; k < K; ++k) sum += expf(load_scalar(m_item + k) - mx);
+                inv_sum = 1.0f / sum;
+            }
+            bool nan_pos = false;
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k) {
+                if (k >= K) break;
+                const int2 kt = ktab[k];
+                const float2 d = load_pair(o_item + 2 * k);
+                float m = load_scalar(m_item + k);
+                if (SOFTMAX) m = expf(m - mx) * inv_sum;
+                const float pxf = fmaf(a.offset_scale, d.x, (float)(wo * a.sw - a.pw + kt.y));
+                const float pyf = fmaf(a.offset_scale, d.y, (float)(ho * a.sh - a.ph + kt.x));
+                Tap tp{0, 0, 0.0f, 0.0f};
+                const int st = make_tap(pyf, pxf, a.H, a.W, tp);
+                nan_pos |= st < 0;
+                uint4 raw[4];
+                float w[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int y = tp.y0 + (c >> 1), x = tp.x0 + (c & 1);
+                    const bool ok = st > 0 && (unsigned)y < (unsigned)a.H && (unsigned)x < (unsigned)a.W;
+                    w[c] = ok ? ((c >> 1) ? tp.ly : 1.0f - tp.ly) * ((c & 1) ? tp.lx : 1.0f - tp.lx) * m : 0.0f;
+                    raw[c] = ok ? ld_nc16(xb + ((long long)y * a.W + x) * GC) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float f[V];
+                    unpack16<T>(raw[c], f);
+#pragma unroll
+                    for (int v = 0; v < V; ++v) acc[v] = fmaf(w[c], f[v], acc[v]);
+                }
+            }
+            if (nan_pos) {
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[v] = __int_as_float(0x7fc00000);
+            }
+        }
+        if (valid) {
+            // 16-byte chunk of row px inside this K-block's slot, swizzled
+            const int chunk = ((g * a.C) & 63) / V + q;
+            *reinterpret_cast<uint4 *>(slot + px * 128 + ((chunk ^ (px & 7)) << 4)) = pack16<T>(acc);
+        }
+        if (RECORDS) __syncwarp();  // records are rewritten by the next step
+    }
+}
+
+template <typename T, int LPI, bool SOFTMAX, int KMAX, bool RECORDS>
 __global__ void __launch_bounds__(kProjThreads, 1)
     core_forward_proj(const __grid_constant__ CUtensorMap wmap, const ProjParams p) {
-    constexpr int V = Storage<T>::kVec;  // 8 channels per 16-byte chunk
-    constexpr int IPW = 32 / LPI;        // items per warp step
+    constexpr int IPW = 32 / LPI;
     const CoreArgs &a = p.a;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     extern __shared__ unsigned char smem_raw[];
-    // 1024-byte aligned base (the swizzle pattern repeats every 1024 bytes)
+    // 1024-byte aligned base (the swizzle pattern repeats every 1024 bytes):
+    // [B-operand ring: kBSlots x npad_max x 128][weight ring: kWStages x 16 KB]
+    // [records: weights, corners][kernel-point table][barriers, tensor-memory address, abort flag]
     const uint32_t raw_a = smem_u32(smem_raw);
     unsigned char *smem = smem_raw + (((raw_a + 1023u) & ~1023u) - raw_a);
-    unsigned char *btile = smem;                                    // KB x npad_max x 128 bytes
-    unsigned char *wst = btile + (size_t)p.KB * p.npad_max * 128;  // kWStages x kWTileBytes
-    uint64_t *bars = reinterpret_cast<uint64_t *>(wst + kWStages * kWTileBytes);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kWStages + kMaxKBlocks + 3);
+    const int slot_bytes = p.npad_max * 128;
+    unsigned char *bring = smem;
+    unsigned char *wst = bring + (size_t)kBSlots * slot_bytes;
+    unsigned char *rp = wst + kWStages * kWTileBytes;
+    float4 *rec_w = reinterpret_cast<float4 *>(rp) + (warp < kGatherWarps ? warp : 0) * KMAX * IPW;
+    int4 *rec_o = reinterpret_cast<int4 *>(rp + (RECORDS ? kGatherWarps * KMAX * IPW * 16 : 0)) +
+                  (warp < kGatherWarps ? warp : 0) * KMAX * IPW;
+    rp += RECORDS ? kGatherWarps * KMAX * IPW * 32 : 0;
+    int2 *ktab = reinterpret_cast<int2 *>(rp);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ktab + KMAX);
+    constexpr int kBars = 2 * kWStages + 2 * kBSlots + 3;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kBars);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const uint32_t wfull = smem_u32(bars), wempty = wfull + 8 * kWStages;
-    const uint32_t kready = wempty + 8 * kWStages, dfull = kready + 8 * kMaxKBlocks;
-    const uint32_t tempty = dfull + 8, drain = dfull + 16;
-    const uint32_t btile_a = smem_u32(btile), wst_a = smem_u32(wst);
+    const uint32_t kready = wempty + 8 * kWStages, bfree = kready + 8 * kBSlots;
+    const uint32_t dfull = bfree + 8 * kBSlots, tempty = dfull + 8, drain = dfull + 16;
+    const uint32_t bring_a = smem_u32(bring), wst_a = smem_u32(wst);
 
+    for (int k = threadIdx.x; k < a.kh * a.kw; k += blockDim.x)
+        ktab[k] = make_int2((k / a.kw) * a.dh, (k % a.kw) * a.dw);
     if (threadIdx.x == 0) {
         for (int i = 0; i < kWStages; ++i) {
             mbar_init(wfull + 8 * i, 1);
             mbar_init(wempty + 8 * i, 1);
         }
-        for (int i = 0; i < kMaxKBlocks; ++i) mbar_init(kready + 8 * i, kGatherWarps);
+        for (int i = 0; i < kBSlots; ++i) {
+            mbar_init(kready + 8 * i, kGatherWarps);
+            mbar_init(bfree + 8 * i, 1);
+        }
         mbar_init(dfull, 1);
         mbar_init(tempty, kGatherWarps);
         mbar_init(drain, 1);
@@ -236,12 +446,13 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 }
                 tc_fence_after();
                 for (int kb = 0; kb < p.KB && !*abort_flag; ++kb) {
-                    if (!wait_or_abort(kready + 8 * kb, ci & 1, abort_flag)) {
+                    const int t = ci * p.KB + kb, bs = t % kBSlots;
+                    if (!wait_or_abort(kready + 8 * bs, (t / kBSlots) & 1, abort_flag)) {
                         raise_abort(abort_flag, p.err);
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t b_kb = btile_a + (uint32_t)(kb * npad * 128);
+                    const uint32_t b_kb = bring_a + (uint32_t)(bs * slot_bytes);
                     for (int mb = 0; mb < p.MB; ++mb, ++it) {
                         const int s = it % kWStages;
                         if (!wait_or_abort(wfull + 8 * s, (it / kWStages) & 1, abort_flag)) {
@@ -257,6 +468,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                         issued = true;
                         mma_commit(wempty + 8 * s);  // weight stage free once these products are done
                     }
+                    if (*abort_flag) break;
+                    mma_commit(bfree + 8 * bs);  // B slot free once this K-block's products are done
                 }
                 if (*abort_flag) break;
                 mma_commit(dfull);  // accumulators of this chunk complete
@@ -268,100 +481,30 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         }
         __syncwarp();
     } else {
-        // ---- gather warps: core samples into the B operand, then the epilogue
-        const int sub = lane % LPI, slot = lane / LPI;
-        const int K = a.kh * a.kw;
-        const int GC = a.G * a.C;
-        const int gpb = 64 / a.C;  // groups per K-block
-        const T *__restrict__ xg = static_cast<const T *>(a.x);
-        const T *__restrict__ off = static_cast<const T *>(a.offset);
-        const T *__restrict__ msk = static_cast<const T *>(a.mask);
+        // ---- gather warps: core samples into the B ring, then the epilogue
         const T *__restrict__ bias = static_cast<const T *>(p.bias);
         T *__restrict__ out = static_cast<T *>(a.out);
-        for (int ci = 0; ci < n_chunks; ++ci) {
+        bool stop = false;
+        for (int ci = 0; ci < n_chunks && !stop; ++ci) {
             long long c0, c1;
             chunk_range(r0, r1, ci, n_chunks, c0, c1);
             const int n_px = (int)(c1 - c0);
             const int npad = (n_px + 15) & ~15;
             for (int kb = 0; kb < p.KB; ++kb) {
-                const int items = n_px * gpb;
-                for (int base = warp * IPW; base < items; base += kGatherWarps * IPW) {
-                    const int item = base + slot;
-                    if (item < items) {
-                        const int px = item / gpb;
-                        const int g = kb * gpb + (item - px * gpb);
-                        long long t = c0 + px;
-                        const int wo = (int)(t % a.Wo);
-                        t /= a.Wo;
-                        const int ho = (int)(t % a.Ho);
-                        const int b = (int)(t / a.Ho);
-                        const long long mi = (c0 + px) * a.G + g;
-                        const T *o_item = off + mi * K * 2;
-                        const T *m_item = msk + mi * K;
-                        float mx = 0.0f, inv_sum = 1.0f;
-                        if (SOFTMAX) {
-                            mx = -INFINITY;
-                            for (int k = 0; k < K; ++k) mx = fmaxf(mx, load_scalar(m_item + k));
-                            float sum = 0.0f;
-                            for (int k = 0; k < K; ++k) sum += expf(load_scalar(m_item + k) - mx);
-                            inv_sum = 1.0f / sum;
-                        }
-                        float acc[V];
-#pragma unroll
-                        for (int v = 0; v < V; ++v) acc[v] = 0.0f;
-                        bool nan_pos = false;
-                        const T *xb = xg + (long long)b * a.H * a.W * GC + g * a.C + sub * V;
-                        int i = 0, j = 0;
-#pragma unroll
-                        for (int k = 0; k < KMAX; ++k) {
-                            if (k >= K) break;
-                            const int by = ho * a.sh - a.ph + i * a.dh;
-                            const int bx = wo * a.sw - a.pw + j * a.dw;
-                            if (++j == a.kw) {
-                                j = 0;
-                                ++i;
-                            }
-                            const float2 d = load_pair(o_item + 2 * k);
-                            float m = load_scalar(m_item + k);
-                            if (SOFTMAX) m = expf(m - mx) * inv_sum;
-                            const float pxf = fmaf(a.offset_scale, d.x, (float)bx);
-                            const float pyf = fmaf(a.offset_scale, d.y, (float)by);
-                            Tap tp{0, 0, 0.0f, 0.0f};
-                            const int st = make_tap(pyf, pxf, a.H, a.W, tp);
-                            nan_pos |= st < 0;
-                            uint4 raw[4];
-                            float w[4];
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                const int y = tp.y0 + (c >> 1), x = tp.x0 + (c & 1);
-                                const bool ok = st > 0 && y >= 0 && y < a.H && x >= 0 && x < a.W;
-                                w[c] = ok ? ((c >> 1) ? tp.ly : 1.0f - tp.ly) * ((c & 1) ? tp.lx : 1.0f - tp.lx) * m
-                                          : 0.0f;
-                                raw[c] = ok ? ld_nc16(xb + ((long long)y * a.W + x) * GC) : make_uint4(0, 0, 0, 0);
-                            }
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                float f[V];
-                                unpack16<T>(raw[c], f);
-#pragma unroll
-                                for (int v = 0; v < V; ++v) acc[v] = fmaf(w[c], f[v], acc[v]);
-                            }
-                        }
-                        if (nan_pos) {
-#pragma unroll
-                            for (int v = 0; v < V; ++v) acc[v] = __int_as_float(0x7fc00000);
-                        }
-                        // 16-byte chunk of row px inside this K-block, swizzled
-                        const int chunk = ((g * a.C) & 63) / V + sub;
-                        unsigned char *dst =
-                            btile + (size_t)kb * npad * 128 + px * 128 + ((chunk ^ (px & 7)) << 4);
-                        *reinterpret_cast<uint4 *>(dst) = pack16<T>(acc);
-                    }
+                const int t = ci * p.KB + kb, bs = t % kBSlots, use = t / kBSlots;
+                // the products that read this slot's previous K-block are done
+                if (use >= 1 && !wait_or_abort(bfree + 8 * bs, (use - 1) & 1, abort_flag)) {
+                    if (lane == 0) raise_abort(abort_flag, p.err);
+                    stop = true;
+                    break;
                 }
-                fence_proxy_async_smem();  // this thread's tile writes before the tensor core reads
+                gather_kblock<T, LPI, SOFTMAX, KMAX, RECORDS>(p, kb, c0, n_px, warp, lane, bring + bs * slot_bytes,
+                                                               rec_w, rec_o, ktab);
+                fence_proxy_async_smem();  // this thread's slot writes before the tensor core reads
                 __syncwarp();
-                if (lane == 0) mbar_arrive(kready + 8 * kb);
+                if (lane == 0) mbar_arrive(kready + 8 * bs);
             }
+            if (stop) break;
             // ---- epilogue: accumulators -> + bias -> storage type
             if (!wait_or_abort(dfull, ci & 1, abort_flag)) {
                 if (lane == 0) raise_abort(abort_flag, p.err);
@@ -377,9 +520,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                     if (o < p.Cout) {
                         const float bo = bias ? load_scalar(bias + o) : 0.0f;
 #pragma unroll
-                        for (int q = 0; q < 16; ++q) {
-                            const int px = blk * 16 + q;
-                            if (px < n_px) out[(c0 + px) * p.Cout + o] = from_f32<T>(v[q] + bo);
+                        for (int r = 0; r < 16; ++r) {
+                            const int px = blk * 16 + r;
+                            if (px < n_px) out[(c0 + px) * p.Cout + o] = from_f32<T>(v[r] + bo);
                         }
                     }
                 }
@@ -399,24 +542,35 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     }
 }
 
-template <typename T, int LPI, bool SOFTMAX, int KMAX>
+template <typename T, int LPI, bool SOFTMAX, int KMAX, bool RECORDS>
 cudaError_t launch_one(const CUtensorMap &map, const ProjParams &p, size_t smem, cudaStream_t stream) {
-    auto kern = core_forward_proj<T, LPI, SOFTMAX, KMAX>;
+    auto kern = core_forward_proj<T, LPI, SOFTMAX, KMAX, RECORDS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<p.n_cta, kProjThreads, smem, stream>>>(map, p);
     return cudaGetLastError();
 }
 
+// Shared memory of one instance: B ring + weight ring + records + table + barriers, plus alignment slack.
+constexpr size_t proj_smem(int npad_max, int lpi, int kmax, bool records) {
+    return (size_t)kBSlots * npad_max * 128 + (size_t)kWStages * kWTileBytes +
+           (records ? (size_t)kGatherWarps * kmax * (32 / lpi) * 32 : 0) + (size_t)kmax * 8 + 256 + 1024;
+}
+
 template <typename T, int LPI>
-cudaError_t launch_lpi(const CUtensorMap &map, const ProjParams &p, size_t smem, cudaStream_t stream) {
+cudaError_t launch_lpi(const CUtensorMap &map, const ProjParams &p, size_t min_smem, cudaStream_t stream) {
     const int K = p.a.kh * p.a.kw;
+    auto pick = [&](size_t need) { return need > min_smem ? need : min_smem; };
     if (K <= 9) {
-        return p.a.softmax ? launch_one<T, LPI, true, 9>(map, p, smem, stream)
-                           : launch_one<T, LPI, false, 9>(map, p, smem, stream);
+        // records for 2..8 lanes per item; a single-lane item computes its own taps
+        constexpr bool R = LPI >= 2;
+        const size_t smem = pick(proj_smem(p.npad_max, LPI, 9, R));
+        return p.a.softmax ? launch_one<T, LPI, true, 9, R>(map, p, smem, stream)
+                           : launch_one<T, LPI, false, 9, R>(map, p, smem, stream);
     }
-    return p.a.softmax ? launch_one<T, LPI, true, 25>(map, p, smem, stream)
-                       : launch_one<T, LPI, false, 25>(map, p, smem, stream);
+    const size_t smem = pick(proj_smem(p.npad_max, LPI, 25, false));
+    return p.a.softmax ? launch_one<T, LPI, true, 25, false>(map, p, smem, stream)
+                       : launch_one<T, LPI, false, 25, false>(map, p, smem, stream);
 }
 
 template <typename T>
@@ -445,12 +599,10 @@ cudaError_t launch_t(const ProjArgs &pa, cudaStream_t stream) {
     p.tmem_cols = cols;
     p.w_box_rows = pa.Cout < 128 ? pa.Cout : 128;
 
-    // B operand + weight ring + barriers, plus the alignment slack; at least
-    // half an SM's shared memory so that one CTA owns the SM's tensor memory
-    size_t smem = (size_t)p.KB * p.npad_max * 128 + (size_t)kWStages * kWTileBytes + 256 + 1024;
+    // at least half an SM's shared memory, so that one CTA owns the SM's
+    // tensor memory (the largest instance needs about 200 KB)
     const size_t half_sm = (size_t)dev->smem_per_sm / 2 + 1024;
-    if (smem < half_sm) smem = half_sm;
-    if (smem > (size_t)dev->smem_optin) return cudaErrorInvalidConfiguration;
+    if (proj_smem(p.npad_max, 2, 9, true) > (size_t)dev->smem_optin) return cudaErrorInvalidConfiguration;
 
     CUtensorMap map;
     const cuuint64_t dims[2] = {(cuuint64_t)a.G * a.C, (cuuint64_t)pa.Cout};
@@ -462,10 +614,10 @@ cudaError_t launch_t(const ProjArgs &pa, cudaStream_t stream) {
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
     switch (a.C * (int)sizeof(T) / 16) {
-        case 1: return launch_lpi<T, 1>(map, p, smem, stream);
-        case 2: return launch_lpi<T, 2>(map, p, smem, stream);
-        case 4: return launch_lpi<T, 4>(map, p, smem, stream);
-        case 8: return launch_lpi<T, 8>(map, p, smem, stream);
+        case 1: return launch_lpi<T, 1>(map, p, half_sm, stream);
+        case 2: return launch_lpi<T, 2>(map, p, half_sm, stream);
+        case 4: return launch_lpi<T, 4>(map, p, half_sm, stream);
+        case 8: return launch_lpi<T, 8>(map, p, half_sm, stream);
         default: return cudaErrorInvalidValue;
     }
 }
