@@ -153,196 +153,221 @@ __device__ __forceinline__ void chunk_range(long long r0, long long r1, int c, i
 // of at most 128 bytes).
 __device__ __align__(16) unsigned char g_zero_row[128];
 
-// Sampling of one 64-channel K-block of a chunk into its B-operand slot.
+// Work of a chunk: its n_px * G (pixel, group) items in one flat list,
+// K-block by K-block and group-major inside a K-block (pixels fastest), so
+// consecutive items of a warp sample neighbouring pixels of one group.  The
+// list is dealt to the gather warps in steps of IPW items, round-robin, so
+// every warp gets the same number of steps whatever the K-block sizes.
+struct ItemPos {
+    int kb, g, px;
+};
+__device__ __forceinline__ ItemPos item_pos(int item, int n_px, int per_kb, int gpb) {
+    ItemPos r;
+    r.kb = item / per_kb;
+    const int j = item - r.kb * per_kb;
+    const int gl = j / n_px;
+    r.px = j - gl * n_px;
+    r.g = r.kb * gpb + gl;
+    return r;
+}
+
+// Offsets and masks of points k0, k0 + LPI, ... of flat item `item` (the
+// record role's raw taps), loaded one step ahead of their use.
+template <typename T, int LPI, bool SOFTMAX, int NT>
+__device__ __forceinline__ void load_raw(const ProjParams &p, long long c0, int n_px, int per_kb, int total,
+                                         int item, int k0, float *dx, float *dy, float *m) {
+    const CoreArgs &a = p.a;
+    const int K = a.kh * a.kw;
+    const bool valid = item < total;
+    const ItemPos ip = item_pos(valid ? item : 0, n_px, per_kb, 64 / a.C);
+    const long long mi = (c0 + ip.px) * a.G + ip.g;
+    const T *off = static_cast<const T *>(a.offset);
+    const T *msk = static_cast<const T *>(a.mask);
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+        const int k = k0 + j * LPI;
+        dx[j] = dy[j] = 0.0f;
+        m[j] = SOFTMAX ? -INFINITY : 0.0f;
+        if (valid && k < K) {
+            const float2 d = load_pair(off + (mi * K + k) * 2);
+            dx[j] = d.x;
+            dy[j] = d.y;
+            m[j] = load_scalar(msk + mi * K + k);
+        }
+    }
+}
+
+// One step: items [base, base + IPW) of the chunk's flat list, sampled into
+// the B-operand slots of their K-blocks.
 //
-// RECORDS (K <= 9, 2..8 lanes per item): per warp step of IPW items, the
-// lanes first turn every (item, point) into a record in shared memory - the
-// four bilinear weights with the modulation folded in and the four corner
-// pixel indices (-1: outside the map, read from the zero row) - computed
-// once by one lane; then the LPI lanes of each item read the records and
-// gather their 16-byte channel chunks of the four corners through L1.
-// Otherwise every lane of an item computes the taps itself.
-// Items are enumerated group-major (pixels fastest), so consecutive items
-// of a warp sample neighbouring pixels of one group.
-template <typename T, int LPI, bool SOFTMAX, int KMAX, bool RECORDS>
-__device__ __forceinline__ void gather_kblock(const ProjParams &p, int kb, long long c0, int n_px, int warp,
-                                              int lane, unsigned char *slot, float4 *rec_w, int4 *rec_o,
-                                              const int2 *ktab) {
+// RECORDS (K <= 9, 2..8 lanes per item): the lanes first turn every (item,
+// point) into a record in shared memory - the four bilinear weights with the
+// modulation folded in and the four corner pixel indices (-1: outside the
+// map, read from the zero row) - computed once by one lane from the raw
+// taps loaded one step earlier; then the LPI lanes of each item read the
+// records and gather their 16-byte channel chunks of the four corners
+// through L1.  Otherwise every lane of an item computes the taps itself.
+template <typename T, int LPI, bool SOFTMAX, int KMAX, bool RECORDS, int NT>
+__device__ __forceinline__ void gather_step(const ProjParams &p, int ci, long long c0, int n_px, int per_kb,
+                                            int total, int base, int lane, unsigned char *bring, int slot_bytes,
+                                            float4 *rec_w, int4 *rec_o, const int2 *ktab, const float *dx,
+                                            const float *dy, const float *m_raw) {
     constexpr int V = Storage<T>::kVec;
     constexpr int IPW = 32 / LPI;
-    constexpr int NT = (KMAX + LPI - 1) / LPI;  // records per lane and step
     const CoreArgs &a = p.a;
     const int K = a.kh * a.kw;
     const int GC = a.G * a.C;
-    const int gpb = 64 / a.C;  // groups per K-block
+    const int gpb = 64 / a.C;
     const unsigned HoWo = (unsigned)a.Ho * (unsigned)a.Wo;
     const T *__restrict__ xg = static_cast<const T *>(a.x);
-    const T *__restrict__ off = static_cast<const T *>(a.offset);
-    const T *__restrict__ msk = static_cast<const T *>(a.mask);
-    const int items = n_px * gpb;
     const int gi = lane / LPI, q = lane % LPI;  // gather role
-    for (int base = warp * IPW; base < items; base += kGatherWarps * IPW) {
-        // the gather role's item
-        const int item = base + gi;
-        const bool valid = item < items;
-        const int gl = item / n_px, px = item - (item / n_px) * n_px;
-        const int g = kb * gpb + gl;
-        const unsigned pix = (unsigned)(c0 + px);
-        const unsigned b = pix / HoWo;
-        const T *xb = xg + (long long)b * a.H * a.W * GC + g * a.C + q * V;
-        float acc[V];
+    const int item = base + gi;
+    const bool valid = item < total;
+    const ItemPos ip = item_pos(valid ? item : 0, n_px, per_kb, gpb);
+    const unsigned pix = (unsigned)(c0 + ip.px);
+    const unsigned b = pix / HoWo;
+    const T *xb = xg + (long long)b * a.H * a.W * GC + ip.g * a.C + q * V;
+    float acc[V];
 #pragma unroll
-        for (int v = 0; v < V; ++v) acc[v] = 0.0f;
-        if (RECORDS) {
-            // ---- records: lane (ri, k0) builds points k0, k0 + LPI, ... of item ri
-            const int ri = lane % IPW, k0 = lane / IPW;
-            const int item_r = base + ri;
-            const bool valid_r = item_r < items;
-            const int gl_r = item_r / n_px, px_r = item_r - (item_r / n_px) * n_px;
-            const unsigned pix_r = (unsigned)(c0 + px_r);
-            const unsigned rem = pix_r % HoWo;
-            const int ho = (int)(rem / (unsigned)a.Wo), wo = (int)(rem % (unsigned)a.Wo);
-            const long long mi = (long long)pix_r * a.G + kb * gpb + gl_r;
-            float dx[NT], dy[NT], m[NT];
+    for (int v = 0; v < V; ++v) acc[v] = 0.0f;
+    if (RECORDS) {
+        // ---- records: lane (ri, k0) builds points k0, k0 + LPI, ... of item ri
+        const int ri = lane % IPW, k0 = lane / IPW;
+        const int item_r = base + ri;
+        const bool valid_r = item_r < total;
+        const ItemPos ipr = item_pos(valid_r ? item_r : 0, n_px, per_kb, gpb);
+        const unsigned rem = (unsigned)(c0 + ipr.px) % HoWo;
+        const int ho = (int)(rem / (unsigned)a.Wo), wo = (int)(rem % (unsigned)a.Wo);
+        float m[NT];
 #pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                const int k = k0 + j * LPI;
-                dx[j] = dy[j] = 0.0f;
-                m[j] = SOFTMAX ? -INFINITY : 0.0f;
-                if (valid_r && k < K) {
-                    const float2 d = load_pair(off + (mi * K + k) * 2);
-                    dx[j] = d.x;
-                    dy[j] = d.y;
-                    m[j] = load_scalar(msk + mi * K + k);
-                }
-            }
-            if (SOFTMAX) {
-                float mx = -INFINITY;
+        for (int j = 0; j < NT; ++j) m[j] = m_raw[j];
+        if (SOFTMAX) {
+            float mx = -INFINITY;
 #pragma unroll
-                for (int j = 0; j < NT; ++j) mx = fmaxf(mx, m[j]);
+            for (int j = 0; j < NT; ++j) mx = fmaxf(mx, m[j]);
 #pragma unroll
-                for (int o = IPW; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-                float sum = 0.0f;
-#pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    m[j] = (k0 + j * LPI < K && valid_r) ? expf(m[j] - mx) : 0.0f;
-                    sum += m[j];
-                }
-#pragma unroll
-                for (int o = IPW; o < 32; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-                const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
-#pragma unroll
-                for (int j = 0; j < NT; ++j) m[j] *= inv;
-            }
-            const float Hf = (float)a.H, Wf = (float)a.W;
+            for (int o = IPW; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            float sum = 0.0f;
 #pragma unroll
             for (int j = 0; j < NT; ++j) {
-                const int k = k0 + j * LPI;
-                if (k >= K) continue;
-                const int2 kt = ktab[k];
-                const float pxf = fmaf(a.offset_scale, dx[j], (float)(wo * a.sw - a.pw + kt.y));
-                const float pyf = fmaf(a.offset_scale, dy[j], (float)(ho * a.sh - a.ph + kt.x));
-                const float fy = floorf(pyf), fx = floorf(pxf);
-                const float ly = pyf - fy, lx = pxf - fx;  // NaN for a NaN position
-                const bool nanp = (pxf != pxf) | (pyf != pyf);
-                const bool inmap = (pyf > -1.0f) & (pyf < Hf) & (pxf > -1.0f) & (pxf < Wf);
-                const int y0 = inmap ? (int)fy : -2, x0 = inmap ? (int)fx : -2;
-                const bool vy0 = (unsigned)y0 < (unsigned)a.H, vy1 = (unsigned)(y0 + 1) < (unsigned)a.H;
-                const bool vx0 = (unsigned)x0 < (unsigned)a.W, vx1 = (unsigned)(x0 + 1) < (unsigned)a.W;
-                const int r00 = y0 * a.W + x0;
-                int4 o4 = make_int4(vy0 & vx0 ? r00 : -1, vy0 & vx1 ? r00 + 1 : -1, vy1 & vx0 ? r00 + a.W : -1,
-                                    vy1 & vx1 ? r00 + a.W + 1 : -1);
-                const float mk = m[j];
-                const float tx0 = (1.0f - lx) * mk, tx1 = lx * mk;
-                float4 w4 = make_float4(fmaf(-tx0, ly, tx0), fmaf(-tx1, ly, tx1), tx0 * ly, tx1 * ly);
-                if (!(valid_r & (inmap | nanp))) w4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                if (!valid_r) o4 = make_int4(-1, -1, -1, -1);
-                rec_w[k * IPW + ri] = w4;  // a NaN position keeps NaN weights and zero-row corners
-                rec_o[k * IPW + ri] = o4;
+                m[j] = (k0 + j * LPI < K && valid_r) ? expf(m[j] - mx) : 0.0f;
+                sum += m[j];
             }
-            __syncwarp();
-            // ---- gather
-            const unsigned char *zrow = g_zero_row + q * 16;
 #pragma unroll
-            for (int k = 0; k < KMAX; ++k) {
-                if (k >= K) break;
-                const float4 w = rec_w[k * IPW + gi];
-                const int4 o = rec_o[k * IPW + gi];
-                const uint4 v0 = ld_nc16(o.x >= 0 ? (const void *)(xb + (long long)o.x * GC) : (const void *)zrow);
-                const uint4 v1 = ld_nc16(o.y >= 0 ? (const void *)(xb + (long long)o.y * GC) : (const void *)zrow);
-                const uint4 v2 = ld_nc16(o.z >= 0 ? (const void *)(xb + (long long)o.z * GC) : (const void *)zrow);
-                const uint4 v3 = ld_nc16(o.w >= 0 ? (const void *)(xb + (long long)o.w * GC) : (const void *)zrow);
+            for (int o = IPW; o < 32; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+#pragma unroll
+            for (int j = 0; j < NT; ++j) m[j] *= inv;
+        }
+        const float Hf = (float)a.H, Wf = (float)a.W;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            const int k = k0 + j * LPI;
+            if (k >= K) continue;
+            const int2 kt = ktab[k];
+            const float pxf = fmaf(a.offset_scale, dx[j], (float)(wo * a.sw - a.pw + kt.y));
+            const float pyf = fmaf(a.offset_scale, dy[j], (float)(ho * a.sh - a.ph + kt.x));
+            const float fy = floorf(pyf), fx = floorf(pxf);
+            const float ly = pyf - fy, lx = pxf - fx;  // NaN for a NaN position
+            const bool nanp = (pxf != pxf) | (pyf != pyf);
+            const bool inmap = (pyf > -1.0f) & (pyf < Hf) & (pxf > -1.0f) & (pxf < Wf);
+            const int y0 = inmap ? (int)fy : -2, x0 = inmap ? (int)fx : -2;
+            const bool vy0 = (unsigned)y0 < (unsigned)a.H, vy1 = (unsigned)(y0 + 1) < (unsigned)a.H;
+            const bool vx0 = (unsigned)x0 < (unsigned)a.W, vx1 = (unsigned)(x0 + 1) < (unsigned)a.W;
+            const int r00 = y0 * a.W + x0;
+            int4 o4 = make_int4(vy0 & vx0 ? r00 : -1, vy0 & vx1 ? r00 + 1 : -1, vy1 & vx0 ? r00 + a.W : -1,
+                                vy1 & vx1 ? r00 + a.W + 1 : -1);
+            const float mk = m[j];
+            const float tx0 = (1.0f - lx) * mk, tx1 = lx * mk;
+            float4 w4 = make_float4(fmaf(-tx0, ly, tx0), fmaf(-tx1, ly, tx1), tx0 * ly, tx1 * ly);
+            if (!(valid_r & (inmap | nanp))) w4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (!valid_r) o4 = make_int4(-1, -1, -1, -1);
+            rec_w[k * IPW + ri] = w4;  // a NaN position keeps NaN weights and zero-row corners
+            rec_o[k * IPW + ri] = o4;
+        }
+        __syncwarp();
+        // ---- gather
+        const unsigned char *zrow = g_zero_row + q * 16;
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            if (k >= K) break;
+            const float4 w = rec_w[k * IPW + gi];
+            const int4 o = rec_o[k * IPW + gi];
+            const uint4 v0 = ld_nc16(o.x >= 0 ? (const void *)(xb + (long long)o.x * GC) : (const void *)zrow);
+            const uint4 v1 = ld_nc16(o.y >= 0 ? (const void *)(xb + (long long)o.y * GC) : (const void *)zrow);
+            const uint4 v2 = ld_nc16(o.z >= 0 ? (const void *)(xb + (long long)o.z * GC) : (const void *)zrow);
+            const uint4 v3 = ld_nc16(o.w >= 0 ? (const void *)(xb + (long long)o.w * GC) : (const void *)zrow);
+            float f[V];
+            unpack16<T>(v0, f);
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] = fmaf(w.x, f[v], acc[v]);
+            unpack16<T>(v1, f);
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] = fmaf(w.y, f[v], acc[v]);
+            unpack16<T>(v2, f);
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] = fmaf(w.z, f[v], acc[v]);
+            unpack16<T>(v3, f);
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] = fmaf(w.w, f[v], acc[v]);
+        }
+    } else if (valid) {
+        // ---- every lane computes the taps of its item
+        const unsigned rem = pix % HoWo;
+        const int ho = (int)(rem / (unsigned)a.Wo), wo = (int)(rem % (unsigned)a.Wo);
+        const long long mi = (long long)pix * a.G + ip.g;
+        const T *o_item = static_cast<const T *>(a.offset) + mi * K * 2;
+        const T *m_item = static_cast<const T *>(a.mask) + mi * K;
+        float mx = 0.0f, inv_sum = 1.0f;
+        if (SOFTMAX) {
+            mx = -INFINITY;
+            for (int k = 0; k < K; ++k) mx = fmaxf(mx, load_scalar(m_item + k));
+            float sum = 0.0f;
+            for (int k = 0; k < K; ++k) sum += expf(load_scalar(m_item + k) - mx);
+            inv_sum = 1.0f / sum;
+        }
+        bool nan_pos = false;
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            if (k >= K) break;
+            const int2 kt = ktab[k];
+            const float2 d = load_pair(o_item + 2 * k);
+            float m = load_scalar(m_item + k);
+            if (SOFTMAX) m = expf(m - mx) * inv_sum;
+            const float pxf = fmaf(a.offset_scale, d.x, (float)(wo * a.sw - a.pw + kt.y));
+            const float pyf = fmaf(a.offset_scale, d.y, (float)(ho * a.sh - a.ph + kt.x));
+            Tap tp{0, 0, 0.0f, 0.0f};
+            const int st = make_tap(pyf, pxf, a.H, a.W, tp);
+            nan_pos |= st < 0;
+            uint4 raw[4];
+            float w[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int y = tp.y0 + (c >> 1), x = tp.x0 + (c & 1);
+                const bool ok = st > 0 && (unsigned)y < (unsigned)a.H && (unsigned)x < (unsigned)a.W;
+                w[c] = ok ? ((c >> 1) ? tp.ly : 1.0f - tp.ly) * ((c & 1) ? tp.lx : 1.0f - tp.lx) * m : 0.0f;
+                raw[c] = ok ? ld_nc16(xb + ((long long)y * a.W + x) * GC) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
                 float f[V];
-                unpack16<T>(v0, f);
+                unpack16<T>(raw[c], f);
 #pragma unroll
-                for (int v = 0; v < V; ++v) acc[v] = fmaf(w.x, f[v], acc[v]);
-                unpack16<T>(v1, f);
-#pragma unroll
-                for (int v = 0; v < V; ++v) acc[v] = fmaf(w.y, f[v], acc[v]);
-                unpack16<T>(v2, f);
-#pragma unroll
-                for (int v = 0; v < V; ++v) acc[v] = fmaf(w.z, f[v], acc[v]);
-                unpack16<T>(v3, f);
-#pragma unroll
-                for (int v = 0; v < V; ++v) acc[v] = fmaf(w.w, f[v], acc[v]);
-            }
-        } else if (valid) {
-            // ---- every lane computes the taps of its item
-            const unsigned rem = pix % HoWo;
-            const int ho = (int)(rem / (unsigned)a.Wo), wo = (int)(rem % (unsigned)a.Wo);
-            const long long mi = (long long)pix * a.G + g;
-            const T *o_item = off + mi * K * 2;
-            const T *m_item = msk + mi * K;
-            float mx = 0.0f, inv_sum = 1.0f;
-            if (SOFTMAX) {
-                mx = -INFINITY;
-                for (int k = 0; k < K; ++k) mx = fmaxf(mx, load_scalar(m_item + k));
-                float sum = 0.0f;
-                for (int k = 0; k < K; ++k) sum += expf(load_scalar(m_item + k) - mx);
-                inv_sum = 1.0f / sum;
-            }
-            bool nan_pos = false;
-#pragma unroll
-            for (int k = 0; k < KMAX; ++k) {
-                if (k >= K) break;
-                const int2 kt = ktab[k];
-                const float2 d = load_pair(o_item + 2 * k);
-                float m = load_scalar(m_item + k);
-                if (SOFTMAX) m = expf(m - mx) * inv_sum;
-                const float pxf = fmaf(a.offset_scale, d.x, (float)(wo * a.sw - a.pw + kt.y));
-                const float pyf = fmaf(a.offset_scale, d.y, (float)(ho * a.sh - a.ph + kt.x));
-                Tap tp{0, 0, 0.0f, 0.0f};
-                const int st = make_tap(pyf, pxf, a.H, a.W, tp);
-                nan_pos |= st < 0;
-                uint4 raw[4];
-                float w[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int y = tp.y0 + (c >> 1), x = tp.x0 + (c & 1);
-                    const bool ok = st > 0 && (unsigned)y < (unsigned)a.H && (unsigned)x < (unsigned)a.W;
-                    w[c] = ok ? ((c >> 1) ? tp.ly : 1.0f - tp.ly) * ((c & 1) ? tp.lx : 1.0f - tp.lx) * m : 0.0f;
-                    raw[c] = ok ? ld_nc16(xb + ((long long)y * a.W + x) * GC) : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float f[V];
-                    unpack16<T>(raw[c], f);
-#pragma unroll
-                    for (int v = 0; v < V; ++v) acc[v] = fmaf(w[c], f[v], acc[v]);
-                }
-            }
-            if (nan_pos) {
-#pragma unroll
-                for (int v = 0; v < V; ++v) acc[v] = __int_as_float(0x7fc00000);
+                for (int v = 0; v < V; ++v) acc[v] = fmaf(w[c], f[v], acc[v]);
             }
         }
-        if (valid) {
-            // 16-byte chunk of row px inside this K-block's slot, swizzled
-            const int chunk = ((g * a.C) & 63) / V + q;
-            *reinterpret_cast<uint4 *>(slot + px * 128 + ((chunk ^ (px & 7)) << 4)) = pack16<T>(acc);
+        if (nan_pos) {
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[v] = __int_as_float(0x7fc00000);
         }
-        if (RECORDS) __syncwarp();  // records are rewritten by the next step
     }
+    if (valid) {
+        // 16-byte chunk of row px inside its K-block's slot, swizzled
+        unsigned char *slot = bring + ((ci * p.KB + ip.kb) % kBSlots) * slot_bytes;
+        const int chunk = ((ip.g * a.C) & 63) / V + q;
+        *reinterpret_cast<uint4 *>(slot + ip.px * 128 + ((chunk ^ (ip.px & 7)) << 4)) = pack16<T>(acc);
+    }
+    if (RECORDS) __syncwarp();  // records are rewritten by the next step
 }
 
 template <typename T, int LPI, bool SOFTMAX, int KMAX, bool RECORDS>
@@ -482,28 +507,73 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         __syncwarp();
     } else {
         // ---- gather warps: core samples into the B ring, then the epilogue
+        constexpr int NT = (KMAX + LPI - 1) / LPI;
         const T *__restrict__ bias = static_cast<const T *>(p.bias);
         T *__restrict__ out = static_cast<T *>(a.out);
+        const int ri = lane % IPW, k0 = lane / IPW;
         bool stop = false;
         for (int ci = 0; ci < n_chunks && !stop; ++ci) {
             long long c0, c1;
             chunk_range(r0, r1, ci, n_chunks, c0, c1);
             const int n_px = (int)(c1 - c0);
             const int npad = (n_px + 15) & ~15;
-            for (int kb = 0; kb < p.KB; ++kb) {
-                const int t = ci * p.KB + kb, bs = t % kBSlots, use = t / kBSlots;
-                // the products that read this slot's previous K-block are done
-                if (use >= 1 && !wait_or_abort(bfree + 8 * bs, (use - 1) & 1, abort_flag)) {
-                    if (lane == 0) raise_abort(abort_flag, p.err);
+            const int per_kb = n_px * (64 / a.C);
+            const int total = per_kb * p.KB;
+            const int n_steps = (total + IPW - 1) / IPW;
+            int waited = -1;    // slots of K-blocks <= waited are known to be free
+            int signaled = 0;   // K-blocks < signaled are handed to the tensor core by this warp
+            // wait until the products that read K-block kb's slot before are done
+            auto slot_free = [&](int kb) -> bool {
+                while (waited < kb) {
+                    ++waited;
+                    const int t = ci * p.KB + waited, use = t / kBSlots;
+                    if (use >= 1 && !wait_or_abort(bfree + 8 * (t % kBSlots), (use - 1) & 1, abort_flag)) {
+                        if (lane == 0) raise_abort(abort_flag, p.err);
+                        return false;
+                    }
+                }
+                return true;
+            };
+            // hand K-blocks [signaled, upto) to the tensor core
+            auto signal = [&](int upto) -> bool {
+                if (upto <= signaled) return true;
+                fence_proxy_async_smem();  // this thread's slot writes before the tensor core reads
+                __syncwarp();
+                for (; signaled < upto; ++signaled) {
+                    // the slot's previous phase is complete before this warp arrives on it again
+                    if (!slot_free(signaled)) return false;
+                    if (lane == 0) mbar_arrive(kready + 8 * ((ci * p.KB + signaled) % kBSlots));
+                }
+                return true;
+            };
+            float dx[NT], dy[NT], m[NT];
+            if (RECORDS) load_raw<T, LPI, SOFTMAX, NT>(p, c0, n_px, per_kb, total, warp * IPW + ri, k0, dx, dy, m);
+            for (int st = warp; st < n_steps; st += kGatherWarps) {
+                const int first = st * IPW;
+                const int last = (first + IPW < total ? first + IPW : total) - 1;
+                if (!slot_free(last / per_kb)) {
                     stop = true;
                     break;
                 }
-                gather_kblock<T, LPI, SOFTMAX, KMAX, RECORDS>(p, kb, c0, n_px, warp, lane, bring + bs * slot_bytes,
-                                                               rec_w, rec_o, ktab);
-                fence_proxy_async_smem();  // this thread's slot writes before the tensor core reads
-                __syncwarp();
-                if (lane == 0) mbar_arrive(kready + 8 * bs);
+                float cdx[NT], cdy[NT], cm[NT];
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    cdx[j] = dx[j];
+                    cdy[j] = dy[j];
+                    cm[j] = m[j];
+                }
+                const int nxt = st + kGatherWarps;
+                if (RECORDS && nxt < n_steps)
+                    load_raw<T, LPI, SOFTMAX, NT>(p, c0, n_px, per_kb, total, nxt * IPW + ri, k0, dx, dy, m);
+                gather_step<T, LPI, SOFTMAX, KMAX, RECORDS, NT>(p, ci, c0, n_px, per_kb, total, first, lane, bring,
+                                                                 slot_bytes, rec_w, rec_o, ktab, cdx, cdy, cm);
+                // every K-block before the one this warp's next step starts in is done
+                if (!signal(nxt < n_steps ? (nxt * IPW) / per_kb : p.KB)) {
+                    stop = true;
+                    break;
+                }
             }
+            if (!stop && !signal(p.KB)) stop = true;
             if (stop) break;
             // ---- epilogue: accumulators -> + bias -> storage type
             if (!wait_or_abort(dfull, ci & 1, abort_flag)) {

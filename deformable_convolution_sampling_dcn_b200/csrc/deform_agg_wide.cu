@@ -163,31 +163,33 @@ __global__ void __launch_bounds__(kAggWarps * 32) agg_forward_pairs_f32(AggArgs 
 
     const float2 *locp = reinterpret_cast<const float2 *>(a.loc);
     float2 uv_next = __ldg(locp + u0);  // unit index == (b*A + anchor)*pairs + pair
+    // (anchor, pair, camera) of the current unit, advanced incrementally
     long long ba = u0 / pairs;
+    int pc = (int)(u0 - ba * pairs);
+    int cam = pc % a.cams;
+    int anchor = (int)(ba % a.A);
+    const float *feat = static_cast<const float *>(a.feat) + (ba / a.A) * a.rows * ROW;
+    bool dirty = false;  // acc holds contributions not yet added to the output
+    auto flush = [&]() {
+        float *o = out + ba * ROW + lane * V;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+            if (nan_pos) {
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[j][v] = __int_as_float(0x7fc00000);
+            }
+            red_add16<float>(o + 32 * j * V, acc[j]);
+#pragma unroll
+            for (int v = 0; v < V; ++v) acc[j][v] = 0.0f;
+        }
+        nan_pos = false;
+        dirty = false;
+    };
     for (long long u = u0; u < u1; ++u) {
         const float2 uv = uv_next;
         if (u + 1 < u1) uv_next = __ldg(locp + u + 1);
-        const long long bau = u / pairs;
-        if (bau != ba) {  // flush the finished anchor
-            float *o = out + ba * ROW + lane * V;
-#pragma unroll
-            for (int j = 0; j < CPL; ++j) {
-                if (nan_pos) {
-#pragma unroll
-                    for (int v = 0; v < V; ++v) acc[j][v] = __int_as_float(0x7fc00000);
-                }
-                red_add16<float>(o + 32 * j * V, acc[j]);
-#pragma unroll
-                for (int v = 0; v < V; ++v) acc[j][v] = 0.0f;
-            }
-            nan_pos = false;
-            ba = bau;
-        }
-        const int pc = (int)(u - bau * pairs);
-        const int cam = pc % a.cams;
-        const int b = (int)(bau / a.A);
-        const float *feat = static_cast<const float *>(a.feat) + (long long)b * a.rows * ROW;
         const long long wbase = u * a.scales;
+        dirty = true;
 #pragma unroll 4
         for (int s = 0; s < a.scales; ++s) {
             const int4 t = tab_smem ? tab[cam * a.scales + s] : load_table(a, cam * a.scales + s);
@@ -201,11 +203,13 @@ __global__ void __launch_bounds__(kAggWarps * 32) agg_forward_pairs_f32(AggArgs 
             for (int j = 0; j < CPL; ++j) w[j] = __ldg(wts + (wbase + s) * a.G + grp[j]);
             float g[4];
             float4 f[4][CPL];
+            const long long row00 = (long long)t.z + (long long)tp.y0 * t.y + tp.x0;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int y = tp.y0 + (c >> 1), x = tp.x0 + (c & 1);
-                const long long row = (long long)t.z + (long long)y * t.y + x;
-                const bool ok = st > 0 && y >= 0 && y < t.x && x >= 0 && x < t.y && row >= 0 && row < a.rows;
+                const long long row = row00 + (c >> 1) * t.y + (c & 1);
+                const bool ok = st > 0 && (unsigned)y < (unsigned)t.x && (unsigned)x < (unsigned)t.y &&
+                                (unsigned long long)row < (unsigned long long)a.rows;
                 g[c] = ok ? ((c >> 1) ? tp.ly : 1.0f - tp.ly) * ((c & 1) ? tp.lx : 1.0f - tp.lx) : 0.0f;
                 const float *r = feat + (ok ? row : 0) * ROW + lane * V;
 #pragma unroll
@@ -225,16 +229,19 @@ __global__ void __launch_bounds__(kAggWarps * 32) agg_forward_pairs_f32(AggArgs 
                     acc[j][3] = fmaf(wg, f[c][j].w, acc[j][3]);
                 }
         }
-    }
-    float *o = out + ba * ROW + lane * V;
-#pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-        if (nan_pos) {
-#pragma unroll
-            for (int v = 0; v < V; ++v) acc[j][v] = __int_as_float(0x7fc00000);
+        // next unit: next pair of this anchor, or the first pair of the next one
+        if (++cam == a.cams) cam = 0;
+        if (++pc == pairs) {
+            flush();
+            pc = 0;
+            ++ba;
+            if (++anchor == a.A) {
+                anchor = 0;
+                feat += (long long)a.rows * ROW;
+            }
         }
-        red_add16<float>(o + 32 * j * V, acc[j]);
     }
+    if (dirty) flush();
 }
 
 template <typename T, int CPL>
