@@ -539,6 +539,51 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+CASES = ("dcnv4_p4", "dcnv3_p3", "dcnv3_p3_dil2", "dcnv4_p4_bwd", "sparse4d", "sparse4d_bwd", "roi_pool",
+         "dcnv4_p4_proj")
+
+
+def run_case(name: str, calls: int) -> None:
+    """Call one workload's entry point `calls` times on cuda:0, untimed (for
+    profilers: `ncu ... python bench.py --case NAME --steps 2`)."""
+    import deformable_convolution_sampling_dcn_b200 as dcn
+
+    dev = torch.device("cuda:0")
+    if name in ("dcnv4_p4", "dcnv3_p3", "dcnv3_p3_dil2"):
+        shape, inp = si.workload_core(name)
+        t = [inp[k].to(dev) for k in ("x", "offset", "mask")]
+        cfg = dict(group=shape.G, kernel=(shape.kh, shape.kw), stride=(shape.stride_h, shape.stride_w),
+                   pad=(shape.pad_h, shape.pad_w), dil=(shape.dil_h, shape.dil_w), softmax=shape.softmax)
+        call = lambda: dcn.dcn_core_forward(*t, **cfg)
+    elif name == "dcnv4_p4_bwd":
+        shape, inp = si.workload_core(name)
+        t = [inp[k].to(dev) for k in ("x", "offset", "mask", "grad_out")]
+        call = lambda: dcn.dcn_core_backward(*t, group=shape.G)
+    elif name in ("sparse4d", "sparse4d_bwd"):
+        bwd = name == "sparse4d_bwd"
+        inp = si.agg_inputs(si.SPARSE4D, si.SEEDS["sparse4d"], with_grad_out=bwd)
+        keys = ("feat", "spatial_shape", "scale_start_index", "sampling_location", "weights")
+        t = [inp[k].to(dev) for k in keys + (("grad_out",) if bwd else ())]
+        call = (lambda: dcn.deform_agg_backward(*t)) if bwd else (lambda: dcn.deform_agg_forward(*t))
+    elif name == "roi_pool":
+        rs = si.ROI_POOL
+        inp = si.roi_inputs(rs, si.SEEDS["roi_pool"])
+        t = [inp[k].to(dev) for k in ("x", "rois", "offset")]
+        call = lambda: dcn.deform_roi_pool_forward(*t, pooled=(rs.PH, rs.PW), sampling=rs.S,
+                                                   spatial_scale=rs.spatial_scale, gamma=rs.gamma)
+    else:
+        shape, inp = si.workload_proj()
+        t = [inp[k].to(dev) for k in ("x", "offset", "mask", "weight", "bias")]
+        call = lambda: dcn.dcn_core_forward_proj(*t, group=shape.G)
+    for _ in range(calls):
+        call()
+    torch.cuda.synchronize()
+    err = dcn._binding.take_device_error()
+    if err:
+        raise SystemExit(f"device error word {err}")
+    print(f"ok {name} x{calls}")
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -549,7 +594,12 @@ def main():
     ap.add_argument("--no-rows", dest="rows", action="store_false")
     ap.add_argument("--no-cpu", dest="cpu", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--case", choices=CASES, default=None,
+                    help="only call this workload's entry point --steps times, untimed (for profilers)")
     args = ap.parse_args()
+    if args.case is not None:
+        run_case(args.case, args.steps)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_env()

@@ -26,7 +26,8 @@ _DTYPE_CODE = {torch.float32: DCN_F32, torch.float16: DCN_F16, torch.bfloat16: D
 # Every entry point include/dcn_b200.h declares.
 EXPORTS = ("dcn_core_output_hw", "dcn_core_forward", "dcn_core_backward", "deform_agg_forward",
            "deform_agg_backward", "dcn_status_string", "dcn_last_error_detail", "dcn_abi_version",
-           "dcn_take_device_error", "deform_roi_pool_forward", "dcn_core_forward_proj")
+           "dcn_take_device_error", "deform_roi_pool_forward", "dcn_core_forward_proj",
+           "dcn_selftest_bounded_wait")
 ABI_VERSION = 1
 
 
@@ -80,6 +81,8 @@ def _declare(lib):
     lib.deform_roi_pool_forward.restype = st
     lib.dcn_core_forward_proj.argtypes = [P, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp]
     lib.dcn_core_forward_proj.restype = st
+    lib.dcn_selftest_bounded_wait.argtypes = [ctypes.c_int32, vp]
+    lib.dcn_selftest_bounded_wait.restype = st
     lib.dcn_take_device_error.argtypes = []
     lib.dcn_take_device_error.restype = ctypes.c_int32
     return lib
@@ -148,6 +151,11 @@ def core_params(x: torch.Tensor, G: int, kernel=(3, 3), stride=(1, 1), pad=(1, 1
 def take_device_error() -> int:
     """Read and clear the device error word (0 = no bounded wait ran out)."""
     return int(lib().dcn_take_device_error())
+
+
+def selftest_bounded_wait(limit_us: int = 2000, device=None) -> None:
+    """Enqueue the bounded-wait self-test on the current stream (see dcn_b200.h)."""
+    check(lib().dcn_selftest_bounded_wait(int(limit_us), torch.cuda.current_stream(device).cuda_stream))
 
 
 def dcn_core_output_hw(p: DcnParams) -> Tuple[int, int]:

@@ -113,6 +113,12 @@ int32_t dcn_take_device_error(void) {
 
 const char *dcn_last_error_detail(void) { return g_detail; }
 
+dcn_status dcn_selftest_bounded_wait(int32_t limit_us, dcn_stream_t stream) {
+    if (limit_us < 1 || limit_us > 10000000) return fail(DCN_ERR_SHAPE, "limit_us must be in [1, 10^7]");
+    return cuda_status(dcnb::launch_bounded_wait_selftest((long long)limit_us * 1000, (cudaStream_t)stream),
+                       "dcn_selftest_bounded_wait launch");
+}
+
 const char *dcn_status_string(dcn_status s) {
     switch (s) {
         case DCN_OK: return "DCN_OK";

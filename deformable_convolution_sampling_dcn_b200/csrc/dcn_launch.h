@@ -70,6 +70,8 @@ cudaError_t launch_core_forward_plane(const CoreArgs &a, cudaStream_t stream, bo
 // Reads and clears the device error word that bounded waits set (bit 0:
 // a TMA wait ran out).  Synchronous.
 cudaError_t take_device_error(unsigned int *value);
+// One thread waits (bounded by limit_ns) on an mbarrier nothing arrives on.
+cudaError_t launch_bounded_wait_selftest(long long limit_ns, cudaStream_t stream);
 // Fused core + projection (tcgen05 GEMM on the core tile in shared memory).
 cudaError_t launch_core_forward_proj(const ProjArgs &a, cudaStream_t stream);
 cudaError_t launch_agg_forward(const AggArgs &a, cudaStream_t stream);

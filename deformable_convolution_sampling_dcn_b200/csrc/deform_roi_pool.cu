@@ -24,17 +24,18 @@ template <typename T, int CPL>
 __global__ void __launch_bounds__(256) roi_pool_forward_kernel(RoiArgs a) {
     constexpr int V = Storage<T>::kVec;
     const int lane = threadIdx.x & 31;
-    const long long bins = (long long)a.N * a.PH * a.PW;
-    const long long bin = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    // N * PH * PW <= 2^31 (checked on the host): 32-bit index arithmetic
+    const unsigned bins = (unsigned)a.N * (unsigned)(a.PH * a.PW);
+    const unsigned bin = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (bin >= bins) return;
-    const int j = (int)(bin % a.PW);
-    const int i = (int)((bin / a.PW) % a.PH);
-    const long long n = bin / ((long long)a.PW * a.PH);
-    const float *r = a.rois + n * 5;
+    const unsigned ij = bin % (unsigned)(a.PH * a.PW);
+    const unsigned n = bin / (unsigned)(a.PH * a.PW);
+    const int i = (int)(ij / (unsigned)a.PW), j = (int)(ij % (unsigned)a.PW);
+    const float *r = a.rois + (long long)n * 5;
     const float rb = __ldg(r);
     const int chunks = a.C / V;
     for (int cb = 0; cb < chunks; cb += 32 * CPL) {
-        T *o = static_cast<T *>(a.out) + bin * a.C + cb * V;
+        T *o = static_cast<T *>(a.out) + (long long)bin * a.C + cb * V;
         const int left = chunks - cb;
         float acc[CPL][V];
 #pragma unroll
@@ -55,37 +56,37 @@ __global__ void __launch_bounds__(256) roi_pool_forward_kernel(RoiArgs a) {
             const float dx = __fmul_rn(__fmul_rn(a.gamma, d.x), rw), dy = __fmul_rn(__fmul_rn(a.gamma, d.y), rh);
             const float bx0 = __fadd_rn(x1, __fmul_rn((float)j, bw)), by0 = __fadd_rn(y1, __fmul_rn((float)i, bh));
             const T *xb = static_cast<const T *>(a.x) + (long long)b * a.H * a.W * a.C + (cb + lane) * V;
-            const int SS = a.S * a.S;
-#pragma unroll 2
-            for (int smp = 0; smp < SS; ++smp) {
-                const int sy = smp / a.S, sx = smp - sy * a.S;
+            for (int sy = 0; sy < a.S; ++sy) {
                 const float py = __fadd_rn(__fadd_rn(by0, __fmul_rn((float)sy + 0.5f, sh)), dy);
-                const float px = __fadd_rn(__fadd_rn(bx0, __fmul_rn((float)sx + 0.5f, sw)), dx);
-                Tap tp{0, 0, 0.0f, 0.0f};
-                const int st = make_tap(py, px, a.H, a.W, tp);
-                nan_pos |= st < 0;
-                float g[4];
-                long long off[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int y = tp.y0 + (c >> 1), x = tp.x0 + (c & 1);
-                    const bool ok = st > 0 && y >= 0 && y < a.H && x >= 0 && x < a.W;
-                    g[c] = ok ? ((c >> 1) ? tp.ly : 1.0f - tp.ly) * ((c & 1) ? tp.lx : 1.0f - tp.lx) : 0.0f;
-                    off[c] = ok ? ((long long)y * a.W + x) * a.C : -1;
-                }
-#pragma unroll
-                for (int q = 0; q < CPL; ++q) {
-                    if (lane + 32 * q >= left) break;
-                    uint4 raw[4];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        raw[c] = off[c] >= 0 ? ld_nc16(xb + off[c] + 32 * q * V) : make_uint4(0, 0, 0, 0);
+#pragma unroll 2
+                for (int sx = 0; sx < a.S; ++sx) {
+                    const float px = __fadd_rn(__fadd_rn(bx0, __fmul_rn((float)sx + 0.5f, sw)), dx);
+                    Tap tp{0, 0, 0.0f, 0.0f};
+                    const int st = make_tap(py, px, a.H, a.W, tp);
+                    nan_pos |= st < 0;
+                    float g[4];
+                    long long off[4];
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        float f[V];
-                        unpack16<T>(raw[c], f);
+                        const int y = tp.y0 + (c >> 1), x = tp.x0 + (c & 1);
+                        const bool ok = st > 0 && y >= 0 && y < a.H && x >= 0 && x < a.W;
+                        g[c] = ok ? ((c >> 1) ? tp.ly : 1.0f - tp.ly) * ((c & 1) ? tp.lx : 1.0f - tp.lx) : 0.0f;
+                        off[c] = ok ? ((long long)y * a.W + x) * a.C : -1;
+                    }
 #pragma unroll
-                        for (int v = 0; v < V; ++v) acc[q][v] = fmaf(g[c], f[v], acc[q][v]);
+                    for (int q = 0; q < CPL; ++q) {
+                        if (lane + 32 * q >= left) break;
+                        uint4 raw[4];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            raw[c] = off[c] >= 0 ? ld_nc16(xb + off[c] + 32 * q * V) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            float f[V];
+                            unpack16<T>(raw[c], f);
+#pragma unroll
+                            for (int v = 0; v < V; ++v) acc[q][v] = fmaf(g[c], f[v], acc[q][v]);
+                        }
                     }
                 }
             }

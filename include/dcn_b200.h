@@ -234,6 +234,15 @@ const char *dcn_last_error_detail(void);
  * 0 after every normal run. */
 int32_t dcn_take_device_error(void);
 
+/* Self-test of the bounded-wait error path above (the pages have no
+ * counterpart; it exists so that the failure path can be exercised without
+ * a fault): enqueues on `stream` one thread that waits on a shared-memory
+ * barrier nothing arrives on, for limit_us microseconds (1 .. 10^7).  The wait
+ * gives up, the kernel sets bit 0 of the device error word and returns; the
+ * next dcn_take_device_error() returns 1 and every later call works as
+ * before.  DCN_ERR_SHAPE for a limit outside the range. */
+dcn_status dcn_selftest_bounded_wait(int32_t limit_us, dcn_stream_t stream);
+
 /* ABI version of this header (bumped on any incompatible change). */
 int32_t dcn_abi_version(void);
 

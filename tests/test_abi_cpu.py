@@ -165,3 +165,8 @@ def test_proj_checks(lib):
         assert f(ctypes.byref(bad), 64, 16, 16, 16, 16, None, 16, None) == B.DCN_ERR_UNSUPPORTED
     empty = params(B=0, G=16, C=32)
     assert f(ctypes.byref(empty), 64, None, None, None, None, None, None, None) == B.DCN_OK
+
+
+def test_selftest_limit_checked_on_host(lib):
+    assert lib.dcn_selftest_bounded_wait(0, None) == B.DCN_ERR_SHAPE
+    assert lib.dcn_selftest_bounded_wait(20_000_000, None) == B.DCN_ERR_SHAPE
