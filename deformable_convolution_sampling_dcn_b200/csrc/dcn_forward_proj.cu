@@ -7,7 +7,7 @@
 // Work split.  The B*Ho*Wo pixels are cut into one contiguous range per CTA
 // (persistent grid, one CTA per SM), processed in chunks of at most 128
 // pixels.  Per chunk:
-//   1. Sixteen gather warps sample the core for every (pixel, group) of the
+//   1. Twenty gather warps sample the core for every (pixel, group) of the
 //      chunk (sub-warp per item, as in the generic kernel), in K-blocks of 64
 //      channels.  Each result is rounded once to the storage type (the value
 //      an unfused core would store) and written straight into shared memory
@@ -38,7 +38,7 @@
 namespace dcnb {
 namespace {
 
-constexpr int kGatherWarps = 16;
+constexpr int kGatherWarps = 20;
 constexpr int kProducerWarp = kGatherWarps;
 constexpr int kMmaWarp = kGatherWarps + 1;
 constexpr int kProjThreads = (kGatherWarps + 2) * 32;
@@ -464,7 +464,11 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             for (int st = warp; st < n_steps; st += kGatherWarps) {
                 const int first = st * IPW;
                 const int last = (first + IPW < total ? first + IPW : total) - 1;
-                if (!slot_free(last / per_kb)) {
+                // K-blocks before this step's first one hold nothing more of this
+                // warp: hand them over before waiting for any slot, so that every
+                // wait below depends only on K-blocks this warp has already
+                // handed over (a step spans at most four K-blocks, the ring size)
+                if (!signal(first / per_kb) || !slot_free(last / per_kb)) {
                     stop = true;
                     break;
                 }

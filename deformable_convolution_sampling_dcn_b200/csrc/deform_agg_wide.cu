@@ -354,13 +354,164 @@ __global__ void __launch_bounds__(kAggWarps * 32) agg_backward_wide(AggArgs a) {
     }
 }
 
+// Backward with pair-granular persistent work (every storage type): warp w
+// of the grid owns the contiguous (anchor, pair) units [U*w/NW, U*(w+1)/NW),
+// so every warp has the same number of samples whatever the anchor count.
+// A unit belongs to exactly one warp, so its location gradient is stored
+// without atomics; the grad_out row is reloaded when the anchor changes.
+// Per sample the four corner rows are loaded first (out-of-map corners load
+// nothing and get weight zero), then the dot products and the 16-byte vector
+// reductions into grad_feat follow.
+template <typename T, int CPL>
+__global__ void __launch_bounds__(kAggWarps * 32) agg_backward_pairs(AggArgs a, long long units, int total_warps) {
+    constexpr int V = Storage<T>::kVec;
+    constexpr int ROW = CPL * 32 * V;
+    __shared__ int4 tab[kAggTableMax];
+    const int lane = threadIdx.x & 31;
+    const int CS = a.cams * a.scales;
+    const bool tab_smem = CS <= kAggTableMax;
+    if (tab_smem)
+        for (int i = threadIdx.x; i < CS; i += blockDim.x) tab[i] = load_table(a, i);
+    __syncthreads();
+
+    const int gw_idx = blockIdx.x * kAggWarps + (threadIdx.x >> 5);
+    const long long u0 = units * gw_idx / total_warps, u1 = units * (gw_idx + 1) / total_warps;
+    if (u0 >= u1) return;
+    const int pairs = a.P * a.cams;
+    const T *__restrict__ wts = static_cast<const T *>(a.weights);
+    T *__restrict__ gw = static_cast<T *>(a.grad_weights);
+    const int gl = a.C / V;  // lanes of one group inside a chunk (a power of two)
+    int grp[CPL];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) grp[j] = (32 * j + lane) * V / a.C;
+
+    long long ba = u0 / pairs;
+    int pc = (int)(u0 - ba * pairs);
+    int cam = pc % a.cams;
+    int anchor = (int)(ba % a.A);
+    long long fofs = (ba / a.A) * a.rows * ROW;
+    float go[CPL][V];
+    auto load_go = [&]() {
+        const T *gout = static_cast<const T *>(a.grad_out) + ba * ROW;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) unpack16<T>(ld_nc16(gout + (32 * j + lane) * V), go[j]);
+    };
+    load_go();
+    for (long long u = u0; u < u1; ++u) {
+        const T *__restrict__ feat = static_cast<const T *>(a.feat) + fofs;
+        T *__restrict__ gfeat = static_cast<T *>(a.grad_feat) + fofs;
+        const float2 uv = __ldg(reinterpret_cast<const float2 *>(a.loc) + u);
+        const long long wbase = u * a.scales;
+        float glx = 0.0f, gly = 0.0f;
+        bool nan_pos = false;
+        for (int s = 0; s < a.scales; ++s) {
+            const int4 t = tab_smem ? tab[cam * a.scales + s] : load_table(a, cam * a.scales + s);
+            const float px = fmaf(uv.x, (float)t.y, -0.5f);
+            const float py = fmaf(uv.y, (float)t.x, -0.5f);
+            Tap tp{0, 0, 0.0f, 0.0f};
+            const int st = make_tap(py, px, t.x, t.y, tp);
+            nan_pos |= st < 0;
+            float w[CPL];
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) w[j] = load_scalar(wts + (wbase + s) * a.G + grp[j]);
+            const float gyv[2] = {1.0f - tp.ly, tp.ly};
+            const float gxv[2] = {1.0f - tp.lx, tp.lx};
+            const long long row00 = (long long)t.z + (long long)tp.y0 * t.y + tp.x0;
+            bool ok[4];
+            long long e0[4];
+            uint4 raw[4][CPL];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int y = tp.y0 + (c >> 1), x = tp.x0 + (c & 1);
+                const long long row = row00 + (c >> 1) * t.y + (c & 1);
+                ok[c] = st > 0 && (unsigned)y < (unsigned)t.x && (unsigned)x < (unsigned)t.y &&
+                        (unsigned long long)row < (unsigned long long)a.rows;
+                e0[c] = (ok[c] ? row : 0) * ROW + lane * V;
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) {
+                    raw[c][j] = make_uint4(0, 0, 0, 0);
+                    if (ok[c]) raw[c][j] = ld_nc16(feat + e0[c] + 32 * j * V);
+                }
+            }
+            float val[CPL], dpx[CPL], dpy[CPL];
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) val[j] = dpx[j] = dpy[j] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int cy = c >> 1, cx = c & 1;
+                const float G = ok[c] ? gyv[cy] * gxv[cx] : 0.0f;
+                const float sx = ok[c] ? (cx ? gyv[cy] : -gyv[cy]) : 0.0f;
+                const float sy = ok[c] ? (cy ? gxv[cx] : -gxv[cx]) : 0.0f;
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) {
+                    float f[V];
+                    unpack16<T>(raw[c][j], f);
+                    float dc = 0.0f;
+#pragma unroll
+                    for (int v = 0; v < V; ++v) dc = fmaf(go[j][v], f[v], dc);
+                    val[j] = fmaf(G, dc, val[j]);
+                    dpx[j] = fmaf(sx, dc, dpx[j]);
+                    dpy[j] = fmaf(sy, dc, dpy[j]);
+                    if (ok[c]) {
+                        const float wg = w[j] * G;
+                        float cv[V];
+#pragma unroll
+                        for (int v = 0; v < V; ++v) cv[v] = wg * go[j][v];
+                        red_add16<T>(gfeat + e0[c] + 32 * j * V, cv);
+                    }
+                }
+            }
+            // weight gradient of (sample, group): sum over the group's lanes
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                float v = val[j];
+                for (int o = 1; o < gl; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (st < 0) v = __int_as_float(0x7fc00000);
+                if ((lane & (gl - 1)) == 0) gw[(wbase + s) * a.G + grp[j]] = from_f32<T>(v);
+                glx = fmaf(w[j] * (float)t.y, dpx[j], glx);
+                gly = fmaf(w[j] * (float)t.x, dpy[j], gly);
+            }
+        }
+        // location gradient of the pair: all groups and scales, one warp
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            glx += __shfl_xor_sync(0xffffffffu, glx, o);
+            gly += __shfl_xor_sync(0xffffffffu, gly, o);
+        }
+        nan_pos = __any_sync(0xffffffffu, nan_pos);
+        if (lane == 0) {
+            const float nan = __int_as_float(0x7fc00000);
+            reinterpret_cast<float2 *>(a.grad_loc)[u] = nan_pos ? make_float2(nan, nan) : make_float2(glx, gly);
+        }
+        // next unit
+        if (++cam == a.cams) cam = 0;
+        if (++pc == pairs) {
+            pc = 0;
+            ++ba;
+            if (++anchor == a.A) {
+                anchor = 0;
+                fofs += (long long)a.rows * ROW;
+            }
+            if (u + 1 < u1) load_go();
+        }
+    }
+}
+
 template <typename T, int CPL>
 cudaError_t launch(const AggArgs &a, bool bwd, cudaStream_t stream) {
     const unsigned grid = (unsigned)((long long)a.B * a.A);
     if (bwd) {
         cudaError_t e = cudaMemsetAsync(a.grad_feat, 0, (size_t)a.B * a.rows * a.G * a.C * sizeof(T), stream);
         if (e != cudaSuccess) return e;
-        agg_backward_wide<T, CPL><<<grid, kAggWarps * 32, 0, stream>>>(a);
+        int dev = 0, sms = 148, per_sm = 1;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, agg_backward_pairs<T, CPL>, kAggWarps * 32, 0);
+        if (per_sm < 1) per_sm = 1;
+        const long long units = (long long)a.B * a.A * a.P * a.cams;
+        long long ctas = (long long)sms * per_sm;
+        if (ctas * kAggWarps > units) ctas = (units + kAggWarps - 1) / kAggWarps;
+        agg_backward_pairs<T, CPL><<<(unsigned)ctas, kAggWarps * 32, 0, stream>>>(a, units, (int)(ctas * kAggWarps));
     } else if (sizeof(T) == 4) {
         // fp32 output: pair-granular persistent warps, partial rows added in L2
         int dev = 0, sms = 148, per_sm = 1;

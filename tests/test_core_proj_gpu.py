@@ -50,6 +50,10 @@ SMALL = [
     (2, 12, 10, 8, 8, 256, "bf16", dict(kh=5, kw=5, pad=2)),       # 25 points, C = 8
     (1, 15, 19, 16, 32, 512, "f16", dict(stride=2, pad=2, dil=2, oob=0.05)),  # strided, dilated, all K-blocks
     (1, 1, 1, 2, 32, 64, "f16", {}),                               # a single output pixel
+    # 20 pixels -> 2 CTAs of 10: the gather warps' first steps start in late
+    # K-blocks, so each must hand over the earlier ones before waiting on a slot
+    (1, 4, 5, 16, 32, 64, "f16", {}),
+    (1, 3, 3, 8, 64, 24, "bf16", {}),                              # 9 pixels, C = 64
 ]
 
 
