@@ -2,23 +2,22 @@
 // deformable_aggregation article, sections 1, 2.1, 2.2 and 4).
 //
 // The sampling position of (anchor, point, camera, scale) does not depend on
-// the group, so one CTA handles one (b, anchor) with all G groups at once:
-// the tap geometry (corner rows, bilinear weights) is computed once per
+// the group, so these kernels handle all G groups of a sample at once: the
+// tap geometry (corner rows, bilinear weights) is computed once per
 // sample instead of once per group, and each bilinear corner of all groups is
 // one contiguous G*C row that the 32 lanes of a warp read as CPL coalesced
 // 512-byte transactions (lane l, chunk j owns elements (32*j + l)*V ...).
-// The CTA's warps split the anchor's (point, camera) pairs; each warp walks
-// the scales of its pairs, and the warps' partial rows are summed through
-// shared memory at the end (forward).  In the backward each pair belongs to
-// exactly one warp, so the location gradient of a pair is reduced inside the
-// warp and stored without atomics; the weight gradient of (sample, group) is
-// reduced over the lanes of the group; the feature gradient is scattered with
-// 16-byte vector reductions.
+// For 16-bit storage the forward runs one CTA per anchor: its warps split the
+// anchor's (point, camera) pairs, each warp walks the scales of its pairs, and
+// the warps' partial rows are summed through shared memory at the end.  The
+// fp32 forward and the backward are persistent and pair-granular (below).  In
+// the backward each pair belongs to exactly one warp, so the location
+// gradient of a pair is reduced inside the warp and stored without atomics;
+// the weight gradient of (sample, group) is reduced over the lanes of the
+// group; the feature gradient is scattered with 16-byte vector reductions.
 //
 // Taken when G*C*sizeof(T) is 512, 1024 or 2048 bytes; other widths use the
-// per-group kernels in deform_agg.cu.  For fp32 outputs the forward uses
-// pair-granular persistent warps (agg_forward_pairs_f32) instead of one CTA
-// per anchor, for load balance.
+// per-group kernels in deform_agg.cu.
 #include "dcn_atomic.cuh"
 #include "dcn_launch.h"
 
@@ -242,116 +241,6 @@ __global__ void __launch_bounds__(kAggWarps * 32) agg_forward_pairs_f32(AggArgs 
         }
     }
     if (dirty) flush();
-}
-
-template <typename T, int CPL>
-__global__ void __launch_bounds__(kAggWarps * 32) agg_backward_wide(AggArgs a) {
-    constexpr int V = Storage<T>::kVec;
-    constexpr int ROW = CPL * 32 * V;
-    __shared__ int4 tab[kAggTableMax];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int CS = a.cams * a.scales;
-    const bool tab_smem = CS <= kAggTableMax;
-    if (tab_smem)
-        for (int i = threadIdx.x; i < CS; i += blockDim.x) tab[i] = load_table(a, i);
-    __syncthreads();
-
-    const long long ba = blockIdx.x;
-    const int b = (int)(ba / a.A);
-    const long long fofs = (long long)b * a.rows * ROW;
-    const T *__restrict__ feat = static_cast<const T *>(a.feat) + fofs;
-    T *__restrict__ gfeat = static_cast<T *>(a.grad_feat) + fofs;
-    const T *__restrict__ wts = static_cast<const T *>(a.weights);
-    T *__restrict__ gw = static_cast<T *>(a.grad_weights);
-    const int pairs = a.P * a.cams;
-    // lanes of one group inside a chunk: C / V consecutive lanes (aligned)
-    const int gl = a.C / V;  // 1..32, a power of two
-    int grp[CPL];
-    float go[CPL][V];
-    const T *gout = static_cast<const T *>(a.grad_out) + ba * ROW;
-#pragma unroll
-    for (int j = 0; j < CPL; ++j) {
-        grp[j] = (32 * j + lane) * V / a.C;
-        unpack16<T>(ld_nc16(gout + (32 * j + lane) * V), go[j]);
-    }
-
-    for (int pc = warp; pc < pairs; pc += kAggWarps) {
-        const int cam = pc % a.cams;
-        const float2 uv = __ldg(reinterpret_cast<const float2 *>(a.loc) + ba * pairs + pc);
-        const long long wbase = (ba * pairs + pc) * a.scales;
-        float glx = 0.0f, gly = 0.0f;
-        bool nan_pos = false;
-        for (int s = 0; s < a.scales; ++s) {
-            const int4 t = tab_smem ? tab[cam * a.scales + s] : load_table(a, cam * a.scales + s);
-            const float px = fmaf(uv.x, (float)t.y, -0.5f);
-            const float py = fmaf(uv.y, (float)t.x, -0.5f);
-            Tap tp{0, 0, 0.0f, 0.0f};
-            const int st = make_tap(py, px, t.x, t.y, tp);
-            float w[CPL];
-#pragma unroll
-            for (int j = 0; j < CPL; ++j) w[j] = load_scalar(wts + (wbase + s) * a.G + grp[j]);
-            float val[CPL], dpx[CPL], dpy[CPL];
-#pragma unroll
-            for (int j = 0; j < CPL; ++j) val[j] = dpx[j] = dpy[j] = 0.0f;
-            if (st > 0) {
-                const float gyv[2] = {1.0f - tp.ly, tp.ly};
-                const float gxv[2] = {1.0f - tp.lx, tp.lx};
-#pragma unroll
-                for (int cy = 0; cy < 2; ++cy) {
-#pragma unroll
-                    for (int cx = 0; cx < 2; ++cx) {
-                        const int y = tp.y0 + cy, x = tp.x0 + cx;
-                        if (y < 0 || y >= t.x || x < 0 || x >= t.y) continue;
-                        const long long row = (long long)t.z + (long long)y * t.y + x;
-                        if (row < 0 || row >= a.rows) continue;
-                        const float G = gyv[cy] * gxv[cx];
-                        const float sx = cx ? gyv[cy] : -gyv[cy];
-                        const float sy = cy ? gxv[cx] : -gxv[cx];
-#pragma unroll
-                        for (int j = 0; j < CPL; ++j) {
-                            const long long e = row * ROW + (32 * j + lane) * V;
-                            float f[V];
-                            unpack16<T>(ld_nc16(feat + e), f);
-                            float dc = 0.0f;
-#pragma unroll
-                            for (int v = 0; v < V; ++v) dc = fmaf(go[j][v], f[v], dc);
-                            val[j] = fmaf(G, dc, val[j]);
-                            dpx[j] = fmaf(sx, dc, dpx[j]);
-                            dpy[j] = fmaf(sy, dc, dpy[j]);
-                            const float wg = w[j] * G;
-                            float c[V];
-#pragma unroll
-                            for (int v = 0; v < V; ++v) c[v] = wg * go[j][v];
-                            red_add16<T>(gfeat + e, c);
-                        }
-                    }
-                }
-            }
-            if (st < 0) nan_pos = true;
-            // weight gradient of (sample, group): sum over the group's lanes
-#pragma unroll
-            for (int j = 0; j < CPL; ++j) {
-                float v = val[j];
-                for (int o = 1; o < gl; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (st < 0) v = __int_as_float(0x7fc00000);
-                if ((lane & (gl - 1)) == 0) gw[(wbase + s) * a.G + grp[j]] = from_f32<T>(v);
-                glx = fmaf(w[j] * (float)t.y, dpx[j], glx);
-                gly = fmaf(w[j] * (float)t.x, dpy[j], gly);
-            }
-        }
-        // location gradient of the pair: all groups and scales, one warp
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            glx += __shfl_xor_sync(0xffffffffu, glx, o);
-            gly += __shfl_xor_sync(0xffffffffu, gly, o);
-        }
-        nan_pos = __any_sync(0xffffffffu, nan_pos);
-        if (lane == 0) {
-            const float nan = __int_as_float(0x7fc00000);
-            reinterpret_cast<float2 *>(a.grad_loc)[ba * pairs + pc] =
-                nan_pos ? make_float2(nan, nan) : make_float2(glx, gly);
-        }
-    }
 }
 
 // Backward with pair-granular persistent work (every storage type): warp w
