@@ -45,13 +45,24 @@ __global__ void __launch_bounds__(256) core_backward_generic(CoreArgs a) {
         const long long item = base + slot;
         const bool active = item < n_items;
         const long long it = active ? item : 0;
-        long long t = it;
-        const int g = (int)(t % a.G);
-        t /= a.G;
-        const int wo = (int)(t % a.Wo);
-        t /= a.Wo;
-        const int ho = (int)(t % a.Ho);
-        const int b = (int)(t / a.Ho);
+        int g, wo, ho, b;
+        if (n_items <= 0xffffffffLL) {  // 32-bit decode (the common case)
+            unsigned t = (unsigned)it;
+            g = (int)(t % (unsigned)a.G);
+            t /= (unsigned)a.G;
+            wo = (int)(t % (unsigned)a.Wo);
+            t /= (unsigned)a.Wo;
+            ho = (int)(t % (unsigned)a.Ho);
+            b = (int)(t / (unsigned)a.Ho);
+        } else {
+            long long t = it;
+            g = (int)(t % a.G);
+            t /= a.G;
+            wo = (int)(t % a.Wo);
+            t /= a.Wo;
+            ho = (int)(t % a.Ho);
+            b = (int)(t / a.Ho);
+        }
         const T *o_item = off + it * K * 2;
         const T *m_item = msk + it * K;
 
@@ -80,36 +91,42 @@ __global__ void __launch_bounds__(256) core_backward_generic(CoreArgs a) {
                 if (SOFTMAX) m = expf(m - mx) * inv_sum;
                 const float px = fmaf(a.offset_scale, d.x, (float)bx);
                 const float py = fmaf(a.offset_scale, d.y, (float)by);
-                Tap tp;
+                Tap tp{0, 0, 0.0f, 0.0f};
                 int st = make_tap(py, px, a.H, a.W, tp);
                 if (!active) st = 0;
                 float val = 0.0f, dpx = 0.0f, dpy = 0.0f;
-                if (st > 0) {
-                    const float gyv[2] = {1.0f - tp.ly, tp.ly};
-                    const float gxv[2] = {1.0f - tp.lx, tp.lx};
-                    const bool vy[2] = {tp.y0 >= 0, tp.y0 + 1 < a.H};
-                    const bool vx[2] = {tp.x0 >= 0, tp.x0 + 1 < a.W};
+                // the four corner rows are loaded first (an out-of-map corner
+                // loads nothing), then the dots and the reductions follow
+                const float gyv[2] = {1.0f - tp.ly, tp.ly};
+                const float gxv[2] = {1.0f - tp.lx, tp.lx};
+                bool ok[4];
+                long long r[4];
+                uint4 raw[4];
 #pragma unroll
-                    for (int cy = 0; cy < 2; ++cy) {
+                for (int c = 0; c < 4; ++c) {
+                    const int y = tp.y0 + (c >> 1), xx = tp.x0 + (c & 1);
+                    ok[c] = st > 0 && (unsigned)y < (unsigned)a.H && (unsigned)xx < (unsigned)a.W;
+                    r[c] = xplane + ((long long)y * a.W + xx) * GC;
+                    raw[c] = ok[c] ? ld_nc16(x + r[c]) : make_uint4(0, 0, 0, 0);
+                }
 #pragma unroll
-                        for (int cx = 0; cx < 2; ++cx) {
-                            if (!(vy[cy] && vx[cx])) continue;
-                            const long long r = xplane + ((long long)(tp.y0 + cy) * a.W + (tp.x0 + cx)) * GC;
-                            float f[V];
-                            unpack16<T>(ld_nc16(x + r), f);
-                            float dc = 0.0f;
+                for (int c = 0; c < 4; ++c) {
+                    const int cy = c >> 1, cx = c & 1;
+                    float f[V];
+                    unpack16<T>(raw[c], f);
+                    float dc = 0.0f;
 #pragma unroll
-                            for (int v = 0; v < V; ++v) dc = fmaf(go[v], f[v], dc);
-                            const float Gc = gyv[cy] * gxv[cx];
-                            val = fmaf(Gc, dc, val);
-                            dpx = fmaf(cx ? gyv[cy] : -gyv[cy], dc, dpx);
-                            dpy = fmaf(cy ? gxv[cx] : -gxv[cx], dc, dpy);
-                            const float mg = m * Gc;
-                            float contrib[V];
+                    for (int v = 0; v < V; ++v) dc = fmaf(go[v], f[v], dc);
+                    const float Gc = ok[c] ? gyv[cy] * gxv[cx] : 0.0f;
+                    val = fmaf(Gc, dc, val);
+                    dpx = fmaf(ok[c] ? (cx ? gyv[cy] : -gyv[cy]) : 0.0f, dc, dpx);
+                    dpy = fmaf(ok[c] ? (cy ? gxv[cx] : -gxv[cx]) : 0.0f, dc, dpy);
+                    if (ok[c]) {
+                        const float mg = m * Gc;
+                        float contrib[V];
 #pragma unroll
-                            for (int v = 0; v < V; ++v) contrib[v] = mg * go[v];
-                            red_add16<T>(gx + r, contrib);
-                        }
+                        for (int v = 0; v < V; ++v) contrib[v] = mg * go[v];
+                        red_add16<T>(gx + r[c], contrib);
                     }
                 }
                 val = subwarp_sum<LPI>(val);
