@@ -5,7 +5,8 @@
 // storage type, so every bilinear corner fetch is one 16-byte load per lane
 // and the LPI lanes of an item together read the C-contiguous corner row.
 // Items are enumerated in output memory order (b, ho, wo, g), so a warp's
-// stores cover consecutive 16-byte chunks.  Out-of-map corners are skipped;
+// stores cover consecutive 16-byte chunks.  Out-of-map corners load nothing
+// and get weight zero (the four corner loads of a tap are issued together);
 // sampling follows the bilinear definition of the DCNv1 page (section 2) and
 // the modulation of the DCNv2 page (section 1) and the YOLOv11 + DCNv4 page
 // (section 1.1: softmax over K for DCNv3, raw for DCNv4).
@@ -33,13 +34,24 @@ __global__ void __launch_bounds__(256) core_forward_generic(CoreArgs a) {
 
     for (long long item = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * IPW + slot;
          item < n_items; item += warps_total * IPW) {
-        long long t = item;
-        const int g = (int)(t % a.G);
-        t /= a.G;
-        const int wo = (int)(t % a.Wo);
-        t /= a.Wo;
-        const int ho = (int)(t % a.Ho);
-        const int b = (int)(t / a.Ho);
+        int g, wo, ho, b;
+        if (n_items <= 0xffffffffLL) {  // 32-bit decode (the common case)
+            unsigned t = (unsigned)item;
+            g = (int)(t % (unsigned)a.G);
+            t /= (unsigned)a.G;
+            wo = (int)(t % (unsigned)a.Wo);
+            t /= (unsigned)a.Wo;
+            ho = (int)(t % (unsigned)a.Ho);
+            b = (int)(t / (unsigned)a.Ho);
+        } else {
+            long long t = item;
+            g = (int)(t % a.G);
+            t /= a.G;
+            wo = (int)(t % a.Wo);
+            t /= a.Wo;
+            ho = (int)(t % a.Ho);
+            b = (int)(t / a.Ho);
+        }
         const T *o_item = off + item * K * 2;
         const T *m_item = msk + item * K;
 
@@ -68,25 +80,28 @@ __global__ void __launch_bounds__(256) core_forward_generic(CoreArgs a) {
                 if (SOFTMAX) m = expf(m - mx) * inv_sum;
                 const float px = fmaf(a.offset_scale, d.x, (float)bx);
                 const float py = fmaf(a.offset_scale, d.y, (float)by);
-                Tap tp;
+                Tap tp{0, 0, 0.0f, 0.0f};
                 const int st = make_tap(py, px, a.H, a.W, tp);
                 if (st < 0) nan_pos = true;
-                if (st <= 0) continue;
+                // the four corner loads are issued together; an out-of-map
+                // corner loads nothing and gets weight zero
                 const float hy = 1.0f - tp.ly, hx = 1.0f - tp.lx;
-                const float w[4] = {hy * hx * m, hy * tp.lx * m, tp.ly * hx * m, tp.ly * tp.lx * m};
-                const bool vy[2] = {tp.y0 >= 0, tp.y0 + 1 < a.H};
-                const bool vx[2] = {tp.x0 >= 0, tp.x0 + 1 < a.W};
+                const float wc[4] = {hy * hx * m, hy * tp.lx * m, tp.ly * hx * m, tp.ly * tp.lx * m};
+                uint4 raw[4];
+                float w[4];
 #pragma unroll
-                for (int cy = 0; cy < 2; ++cy) {
+                for (int c = 0; c < 4; ++c) {
+                    const int y = tp.y0 + (c >> 1), xx = tp.x0 + (c & 1);
+                    const bool ok = st > 0 && (unsigned)y < (unsigned)a.H && (unsigned)xx < (unsigned)a.W;
+                    w[c] = ok ? wc[c] : 0.0f;
+                    raw[c] = ok ? ld_nc16(xb + ((long long)y * a.W + xx) * GC) : make_uint4(0, 0, 0, 0);
+                }
 #pragma unroll
-                    for (int cx = 0; cx < 2; ++cx) {
-                        if (!(vy[cy] && vx[cx])) continue;
-                        const T *p = xb + ((long long)(tp.y0 + cy) * a.W + (tp.x0 + cx)) * GC;
-                        float f[V];
-                        unpack16<T>(ld_nc16(p), f);
+                for (int c = 0; c < 4; ++c) {
+                    float f[V];
+                    unpack16<T>(raw[c], f);
 #pragma unroll
-                        for (int v = 0; v < V; ++v) acc[v] = fmaf(w[cy * 2 + cx], f[v], acc[v]);
-                    }
+                    for (int v = 0; v < V; ++v) acc[v] = fmaf(w[c], f[v], acc[v]);
                 }
             }
         }
