@@ -122,9 +122,9 @@ dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offs
  * result once.  The core never reaches device memory.
  * Supported: fp16 and bf16 (fp32 returns DCN_ERR_UNSUPPORTED), C <= 64 with
  * G*C a multiple of 64 up to 512, kh*kw <= 25, Cout a multiple of 8 in
- * [8, 512], H*W and B*Ho*Wo below 2^31; both mask modes.  x, weight and out 16-byte aligned, offset
- * 4-byte, mask and bias 2-byte.  A NaN sampling position makes every output
- * channel of its pixel NaN.
+ * [8, 512], H*W and B*Ho*Wo below 2^31; both mask modes.  x, weight and out
+ * 16-byte aligned, offset 4-byte, mask and bias 2-byte.  A NaN sampling
+ * position makes every output channel of its pixel NaN.
  */
 dcn_status dcn_core_forward_proj(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
                                  const void *mask, const void *weight, const void *bias, void *out,
@@ -206,7 +206,8 @@ dcn_status deform_agg_backward(const dagg_params *p, const void *feat,
  * + ((s + 0.5) * bin / S) + dp, pixel centres at integers; positions are
  * formed in fp32, one rounding per operation in that order.  A NaN position
  * makes its bin NaN.  C*sizeof(dtype) must be a multiple of 16 bytes (at most
- * 65536 channels); x and out 16-byte aligned, rois/offset 8-byte aligned.
+ * 65536 channels), num_rois*PH*PW at most 2^31; x and out 16-byte aligned,
+ * rois 4-byte, offset 8-byte.
  */
 typedef struct {
     int32_t B, H, W, C;           /* input map */
