@@ -45,7 +45,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 # while these are unchanged.
 KERNEL_SOURCES = [os.path.join(ROOT, "deformable_convolution_sampling_dcn_b200", "csrc", f)
                   for f in ("dcn_forward_plane.cu", "dcn_forward_staged.cuh", "dcn_forward_staged_f16.cu",
-                            "dcn_tma.cuh", "dcn_forward_generic.cu", "dcn_common.cuh")]
+                            "dcn_tma.cuh", "dcn_common.cuh", "dcn_device.h")]
 
 
 def kernel_hash() -> str:
