@@ -137,10 +137,13 @@ struct Tap {
 };
 
 // Returns 1 if the tap may contribute, 0 if every neighbour lies outside the
-// map (or p is infinite), and -1 if p is not a number.
+// map (or p is infinite), and -1 if p is not a number.  The support is
+// floor(p) in [-1, size-1], i.e. -1 <= p < size: at p = -1 exactly the
+// in-map corner has weight zero but, with the derivative taken from the
+// right, a non-zero position gradient.
 __device__ __forceinline__ int make_tap(float py, float px, int H, int W, Tap &t) {
     if (py != py || px != px) return -1;
-    if (!(py > -1.0f && py < (float)H && px > -1.0f && px < (float)W)) return 0;
+    if (!(py >= -1.0f && py < (float)H && px >= -1.0f && px < (float)W)) return 0;
     const float fy = floorf(py), fx = floorf(px);
     t.y0 = (int)fy;
     t.x0 = (int)fx;

@@ -183,7 +183,7 @@ __device__ __forceinline__ void gather_step(const ProjParams &p, int ci, long lo
             const float fy = floorf(pyf), fx = floorf(pxf);
             const float ly = pyf - fy, lx = pxf - fx;  // NaN for a NaN position
             const bool nanp = (pxf != pxf) | (pyf != pyf);
-            const bool inmap = (pyf > -1.0f) & (pyf < Hf) & (pxf > -1.0f) & (pxf < Wf);
+            const bool inmap = (pyf >= -1.0f) & (pyf < Hf) & (pxf >= -1.0f) & (pxf < Wf);
             const int y0 = inmap ? (int)fy : -2, x0 = inmap ? (int)fx : -2;
             const bool vy0 = (unsigned)y0 < (unsigned)a.H, vy1 = (unsigned)(y0 + 1) < (unsigned)a.H;
             const bool vx0 = (unsigned)x0 < (unsigned)a.W, vx1 = (unsigned)(x0 + 1) < (unsigned)a.W;

@@ -292,8 +292,8 @@ __global__ void __launch_bounds__(kStagedMaxThreads, 1)
                     const float fy = floorf(py), fx = floorf(px);
                     const float ly = py - fy, lx = px - fx;  // NaN for a NaN position
                     const bool nanp = (px != px) | (py != py);
-                    // some neighbour inside the map (false for NaN and infinite positions)
-                    const bool inmap = (py > -1.0f) & (py < Hf) & (px > -1.0f) & (px < Wf);
+                    // floor(p) in [-1, size-1] (false for NaN and infinite positions)
+                    const bool inmap = (py >= -1.0f) & (py < Hf) & (px >= -1.0f) & (px < Wf);
                     const int y0 = (int)fy, x0 = (int)fx;  // meaningful only when inmap
                     const bool inband = (unsigned)y0 - (unsigned)sg.ys < (unsigned)(sg.ye - sg.ys);
                     const bool smem_tap = r_ok & inmap & inband;

@@ -445,7 +445,34 @@ def pin_agg_backward(lib):
 
 CORE_PINS = [pin_identity, pin_box_sum, pin_shifted_gather, pin_affine_field, pin_softmax_constant,
              pin_softmax_vs_raw, pin_brute_force]
-BACKWARD_PINS = [pin_backward_fd, pin_backward_autograd]
+def pin_backward_right_derivative_at_minus_one(lib):
+    """At a sampling position exactly on p = -1 the value is zero, and the
+    offset gradient is the derivative from the right (the floor() support
+    convention): it equals the forward difference (L(p + h) - L(p)) / h, which
+    is exact because the interpolation is linear inside the cell [-1, 0)."""
+    rng = np.random.default_rng(301)
+    B, H, W, G, C = 1, 4, 5, 1, 3
+    x = rng.standard_normal((B, H, W, G * C))
+    go = rng.standard_normal((B, H, W, G * C))
+    mask = np.zeros((B, H, W, G, 9))
+    off = np.zeros((B, H, W, G, 9, 2))
+    # output (0, 2), point (0, 1): base (-1, 2) with pad 1; output (2, 0), point (1, 0): base (2, -1)
+    mask[0, 0, 2, 0, 1] = 0.7
+    mask[0, 2, 0, 0, 3] = -1.3
+    geom = (H, W, 3, 3, (1, 1), (1, 1), (1, 1))
+    g = oracle.dcn_backward(x, off, mask, go, G=G, lib=lib)
+    h = 2.0 ** -10
+    L0 = _loss(lib, x, off, mask, go, G, geom, 1.0, False)
+    for (ho, wo, k, axis) in ((0, 2, 1, 1), (2, 0, 3, 0)):
+        o2 = off.copy()
+        o2[0, ho, wo, 0, k, axis] = h
+        fd = (_loss(lib, x, o2, mask, go, G, geom, 1.0, False) - L0) / h
+        an = g["grad_offset"][0, ho, wo, 0, k, axis]
+        assert abs(an) > 1e-3, "right derivative at p = -1 is not zero for this input"
+        assert abs(an - fd) <= 1e-9 * (1 + abs(fd)), f"right derivative at p = -1: {an} vs {fd}"
+
+
+BACKWARD_PINS = [pin_backward_fd, pin_backward_autograd, pin_backward_right_derivative_at_minus_one]
 AGG_PINS = [pin_agg_brute_force, pin_agg_grid_sample, pin_agg_backward]
 ALL_PINS = CORE_PINS + BACKWARD_PINS + AGG_PINS
 

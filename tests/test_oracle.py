@@ -76,6 +76,9 @@ def test_far_offsets_contribute_nothing(oracle_lib):
 # (text to replace, replacement, occurrences to replace (0 = all), pins to run)
 MUTATIONS = [
     ("(float)d[0], (float)bx", "(float)d[1], (float)bx", 0, pins.CORE_PINS),
+    # strict support (-1 < p instead of -1 <= p) in the backward
+    ("if (!(fy >= -1.0 && fy <= H - 1 && fx >= -1.0 && fx <= W - 1)) continue;",
+     "if (!(fy > -1.0 && fy <= H - 1 && fx > -1.0 && fx <= W - 1)) continue;", 0, pins.BACKWARD_PINS),
     ("const int by = ho * sh - ph + i * dh;", "const int by = ho * sh + ph + i * dh;", 0, pins.CORE_PINS),
     ("const int bx = wo * sw - pw + j * dw;", "const int bx = wo * sw - pw + j;", 0, pins.CORE_PINS),
     ("const int by = ho * sh - ph + i * dh;", "const int by = ho - ph + i * dh;", 0, pins.CORE_PINS),
