@@ -71,6 +71,8 @@ def _bind(lib):
     lib.oracle_roi_pool_forward.restype = None
     lib.oracle_pointwise_projection.argtypes = [ctypes.c_longlong, i, i, dp, dp, dp, dp]
     lib.oracle_pointwise_projection.restype = None
+    lib.oracle_deform_conv_forward.argtypes = [i] * 13 + [ctypes.c_float, i, i, dp, dp, dp, dp, dp, dp]
+    lib.oracle_deform_conv_forward.restype = None
     return lib
 
 
@@ -133,6 +135,29 @@ def dcn_forward_proj(x, offset, mask, weight, bias=None, *, G: int, lib=None, **
     """The sampling core followed by its pointwise projection, both in fp64:
     pointwise_projection(dcn_forward(x, offset, mask, ...), weight, bias)."""
     return pointwise_projection(dcn_forward(x, offset, mask, G=G, lib=lib, **core), weight, bias, lib=lib)
+
+
+def deform_conv_forward(x, offset, mask, weight, bias=None, *, G: int, kh: int = 3, kw: int = 3, stride=(1, 1),
+                        pad=(1, 1), dil=(1, 1), offset_scale: float = 1.0, softmax: bool = False,
+                        lib=None) -> np.ndarray:
+    """out [B,Ho,Wo,Cout] in fp64: modulated deformable convolution with weight [Cout, K, G*C]."""
+    lib = lib or load()
+    x, offset, mask, weight = _f64(x), _f64(offset), _f64(mask), _f64(weight)
+    B, H, W, GC = x.shape
+    C = GC // G
+    K = kh * kw
+    Cout = weight.shape[0]
+    assert weight.shape == (Cout, K, GC), weight.shape
+    Ho, Wo = out_hw(H, W, kh, kw, *stride, *pad, *dil)
+    assert offset.shape == (B, Ho, Wo, G, K, 2) and mask.shape == (B, Ho, Wo, G, K)
+    b = None if bias is None else _f64(bias)
+    out = np.empty((B, Ho, Wo, Cout), dtype=np.float64)
+    lib.oracle_deform_conv_forward(B, H, W, G, C, kh, kw, stride[0], stride[1], pad[0], pad[1], dil[0], dil[1],
+                                   float(offset_scale), int(bool(softmax)), Cout, _ptr(x, ctypes.c_double),
+                                   _ptr(offset, ctypes.c_double), _ptr(mask, ctypes.c_double),
+                                   _ptr(weight, ctypes.c_double), None if b is None else _ptr(b, ctypes.c_double),
+                                   _ptr(out, ctypes.c_double))
+    return out
 
 
 def dcn_backward(x, offset, mask, grad_out, *, G: int, kh: int = 3, kw: int = 3, stride=(1, 1),

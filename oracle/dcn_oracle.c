@@ -28,7 +28,9 @@
  *   article, sections 1, 2.1 and 2.2).
  *
  *   The pointwise projection (1x1 convolution with bias) that follows the
- *   core in the DCNv4 module (YOLOv11 + DCNv4 article, section 3.2).
+ *   core in the DCNv4 module (YOLOv11 + DCNv4 article, section 3.2), and the
+ *   modulated deformable convolution with a dense weight per kernel point
+ *   (DCNv2 page, section 1; DCNv1 page, section 1).
  *
  * Readings where the pages are silent (each one is listed in the design notes):
  *   - base grid point of kernel point (i,j) at output (ho,wo):
@@ -175,6 +177,81 @@ void oracle_pointwise_projection(long long npix, int Cin, int Cout, const double
             y[o] = s;
         }
     }
+}
+
+/*
+ * Modulated deformable convolution (DCNv2: "DCNv2实战：在YOLOv5中替换普通卷积..."
+ * section 1, y(p0) = sum_n w(pn) * x(p0 + pn + dpn) * dm_n; DCNv1 page, section 1,
+ * without the modulation): every kernel point k has its own dense weight
+ * w_k[o, c] over the input channels,
+ *     out[p, o] = bias[o] + sum_k sum_j weight[o, k, j] * m_k * x_j(p + p_k + dp_k),
+ * j = g*C + c over the G*C input channels, the offset and modulation of point
+ * k shared by the C channels of deformable group g (the same offset/mask
+ * tensors and sampling as the core above).  weight is [Cout, K, G*C]; bias
+ * may be NULL.  The sampled, modulated values of one output pixel are formed
+ * first (K*G*C of them), then contracted with the weight.
+ */
+void oracle_deform_conv_forward(int B, int H, int W, int G, int C, int kh, int kw,
+                                int sh, int sw, int ph, int pw, int dh, int dw,
+                                float offset_scale, int softmax, int Cout,
+                                const double *x, const double *offset, const double *mask,
+                                const double *weight, const double *bias, double *out)
+{
+    const int K = kh * kw;
+    const int GC = G * C;
+    const int Ho = (H + 2 * ph - (dh * (kh - 1) + 1)) / sh + 1;
+    const int Wo = (W + 2 * pw - (dw * (kw - 1) + 1)) / sw + 1;
+
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b)
+        for (int ho = 0; ho < Ho; ++ho) {
+            double *col = (double *)malloc(sizeof(double) * (size_t)K * GC);
+            double *m = (double *)malloc(sizeof(double) * (size_t)K);
+            for (int wo = 0; wo < Wo; ++wo) {
+                for (int t = 0; t < K * GC; ++t) col[t] = 0.0;
+                for (int g = 0; g < G; ++g) {
+                    const size_t item = (((size_t)b * Ho + ho) * Wo + wo) * G + g;
+                    modulation(mask + item * K, K, softmax, m);
+                    for (int i = 0; i < kh; ++i)
+                        for (int j = 0; j < kw; ++j) {
+                            const int k = i * kw + j;
+                            double *ck = col + (size_t)k * GC + (size_t)g * C;
+                            const int by = ho * sh - ph + i * dh;
+                            const int bx = wo * sw - pw + j * dw;
+                            const double *d = offset + (item * K + k) * 2;
+                            const float px = fmaf(offset_scale, (float)d[0], (float)bx);
+                            const float py = fmaf(offset_scale, (float)d[1], (float)by);
+                            if (isnan(px) || isnan(py)) {
+                                for (int c = 0; c < C; ++c) ck[c] = NAN;
+                                continue;
+                            }
+                            const double fy = floor((double)py), fx = floor((double)px);
+                            if (!(fy >= -1.0 && fy <= H - 1 && fx >= -1.0 && fx <= W - 1)) continue;
+                            const int y0 = (int)fy, x0 = (int)fx;
+                            for (int qy = y0; qy <= y0 + 1; ++qy) {
+                                if (qy < 0 || qy >= H) continue;
+                                const double gy = g_kernel(qy, py);
+                                for (int qx = x0; qx <= x0 + 1; ++qx) {
+                                    if (qx < 0 || qx >= W) continue;
+                                    const double Gq = g_kernel(qx, px) * gy;
+                                    const double *xq = x + (((size_t)b * H + qy) * W + qx) * (size_t)GC
+                                                         + (size_t)g * C;
+                                    for (int c = 0; c < C; ++c) ck[c] += m[k] * Gq * xq[c];
+                                }
+                            }
+                        }
+                }
+                double *y = out + (((size_t)b * Ho + ho) * Wo + wo) * (size_t)Cout;
+                for (int o = 0; o < Cout; ++o) {
+                    const double *w = weight + (size_t)o * K * GC;
+                    double acc = bias ? bias[o] : 0.0;
+                    for (int t = 0; t < K * GC; ++t) acc += w[t] * col[t];
+                    y[o] = acc;
+                }
+            }
+            free(col);
+            free(m);
+        }
 }
 
 /*

@@ -623,3 +623,61 @@ def pin_proj_composed_identity(lib):
 
 PROJ_PINS = [pin_proj_conv2d, pin_proj_closed_forms, pin_proj_composed_identity]
 ALL_PINS = ALL_PINS + PROJ_PINS
+
+
+# ---------------------------------------------------------------- modulated deformable convolution pins
+def _dconv_case(seed, B=2, H=7, W=9, G=2, C=3, cout=5, kh=3, kw=3):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, H, W, G * C)), rng.standard_normal((cout, kh * kw, G * C)),
+            rng.standard_normal(cout))
+
+
+def _tv_offset_mask(off, mask):
+    """ours: offset [B,Ho,Wo,G,K,(dx,dy)], mask [B,Ho,Wo,G,K] -> torchvision's
+    offset [B, 2*G*K, Ho, Wo] with (dy, dx) per (g, k), mask [B, G*K, Ho, Wo]."""
+    B, Ho, Wo, G, K, _ = off.shape
+    tv_off = np.stack([off[..., 1], off[..., 0]], axis=-1).reshape(B, Ho, Wo, G * K * 2).transpose(0, 3, 1, 2)
+    tv_mask = mask.reshape(B, Ho, Wo, G * K).transpose(0, 3, 1, 2)
+    return torch.from_numpy(np.ascontiguousarray(tv_off)), torch.from_numpy(np.ascontiguousarray(tv_mask))
+
+
+def pin_dconv_torchvision(lib):
+    """Equals torchvision's deform_conv2d (DCNv2 with mask) on several geometries;
+    offsets on a 1/256 lattice so the fp32 positions are exact."""
+    from torchvision.ops import deform_conv2d
+
+    for n, (kh, kw, stride, pad, dil) in enumerate([(3, 3, (1, 1), (1, 1), (1, 1)), (3, 2, (2, 1), (1, 0), (1, 2)),
+                                                    (1, 3, (1, 2), (0, 2), (2, 1))]):
+        x, w, b = _dconv_case(400 + n, kh=kh, kw=kw)
+        B, H, W, GC = x.shape
+        G = 2
+        Ho, Wo = oracle.out_hw(H, W, kh, kw, *stride, *pad, *dil)
+        rng = np.random.default_rng(410 + n)
+        off = np.round(rng.standard_normal((B, Ho, Wo, G, kh * kw, 2)) * 1.5 * 256) / 256
+        mask = rng.uniform(0.0, 1.0, (B, Ho, Wo, G, kh * kw))
+        out = oracle.deform_conv_forward(x, off, mask, w, b, G=G, kh=kh, kw=kw, stride=stride, pad=pad, dil=dil,
+                                         lib=lib)
+        tv_off, tv_mask = _tv_offset_mask(off, mask)
+        tv_w = torch.from_numpy(w.reshape(w.shape[0], kh, kw, GC).transpose(0, 3, 1, 2).copy())
+        ref = deform_conv2d(torch.from_numpy(x).permute(0, 3, 1, 2).contiguous(), tv_off, tv_w, torch.from_numpy(b),
+                            stride=stride, padding=pad, dilation=dil, mask=tv_mask)
+        assert np.allclose(out, ref.permute(0, 2, 3, 1).numpy(), rtol=0, atol=1e-10), f"deform conv vs torchvision {n}"
+
+
+def pin_dconv_regular_conv(lib):
+    """Zero offsets and unit modulation reduce it to an ordinary convolution."""
+    x, w, b = _dconv_case(420, B=2, H=8, W=6, G=3, C=2, cout=4)
+    B, H, W, GC = x.shape
+    for stride, pad, dil in [((1, 1), (1, 1), (1, 1)), ((2, 1), (2, 0), (2, 1))]:
+        Ho, Wo = oracle.out_hw(H, W, 3, 3, *stride, *pad, *dil)
+        off = np.zeros((B, Ho, Wo, 3, 9, 2))
+        mask = np.ones((B, Ho, Wo, 3, 9))
+        out = oracle.deform_conv_forward(x, off, mask, w, b, G=3, stride=stride, pad=pad, dil=dil, lib=lib)
+        ref = torch.nn.functional.conv2d(torch.from_numpy(x).permute(0, 3, 1, 2),
+                                         torch.from_numpy(w.reshape(4, 3, 3, GC).transpose(0, 3, 1, 2).copy()),
+                                         torch.from_numpy(b), stride=stride, padding=pad, dilation=dil)
+        assert np.allclose(out, ref.permute(0, 2, 3, 1).numpy(), rtol=0, atol=1e-11), "deform conv vs conv2d"
+
+
+DCONV_PINS = [pin_dconv_torchvision, pin_dconv_regular_conv]
+ALL_PINS = ALL_PINS + DCONV_PINS

@@ -115,6 +115,11 @@ MUTATIONS = [
      "            for (int c = 0; c < Cin; ++c) s += w[c] * v[c];",
      "const double *w = Wt + (size_t)o;\n            double s = bias ? bias[o] : 0.0;\n"
      "            for (int c = 0; c < Cin; ++c) s += w[(size_t)c * Cout] * v[c];", 0, pins.PROJ_PINS),
+    ("double *ck = col + (size_t)k * GC + (size_t)g * C;", "double *ck = col + (size_t)g * K * C + (size_t)k * C;",
+     0, pins.DCONV_PINS),
+    ("for (int c = 0; c < C; ++c) ck[c] += m[k] * Gq * xq[c];", "for (int c = 0; c < C; ++c) ck[c] += Gq * xq[c];",
+     0, pins.DCONV_PINS),
+    ("double acc = bias ? bias[o] : 0.0;", "double acc = 0.0;", 0, pins.DCONV_PINS),
     ("double s = bias ? bias[o] : 0.0;", "double s = 0.0;", 0, pins.PROJ_PINS),
     ("double s = bias ? bias[o] : 0.0;", "double s = bias ? bias[0] : 0.0;", 0, pins.PROJ_PINS),
 ]
