@@ -494,7 +494,32 @@ def measure_rows(dcn, dev, stream, l2, barrier, world, steps=280):
     out["dcnv4_p4_proj"] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(shape.samples / ms / 1e6, 2),
                             "GB_s": round(pbytes / ms / 1e6, 1), "gemm_TFLOP_s": round(flops / ms / 1e9, 1),
                             "unfused_core_then_cublas_us": round(ms_u * 1e3, 2), "Cout": cout, "R": R}
+    del sets
+
+    # modulated deformable convolution (a dense weight per kernel point) at the
+    # P4 shape, 512 -> 512, fp16
+    shape, inp = workload_deform_conv()
+    t = [inp[k].to(dev) for k in ("x", "offset", "mask", "weight", "bias")]
+    cout = t[3].shape[0]
+    R = max(2, math.ceil(4 * l2 / pbytes))
+    sets = [[u.clone() for u in t] + [torch.empty((shape.B, shape.Ho, shape.Wo, cout), dtype=t[0].dtype, device=dev)]
+            for _ in range(R)]
+
+    def mkd(s):
+        return lambda: dcn.dcn_deform_conv_forward(s[0], s[1], s[2], s[3], s[4], group=shape.G, out=s[5])
+
+    ms = time_steps(mkd, sets, steps, 3 * R, stream, barrier, world) / steps
+    flops = 2.0 * shape.B * shape.Ho * shape.Wo * cout * shape.K * shape.G * shape.C
+    out["dcnv2_p4_deform_conv"] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(shape.samples / ms / 1e6, 2),
+                                   "gemm_TFLOP_s": round(flops / ms / 1e9, 1), "Cout": cout, "R": R}
     return out
+
+
+def workload_deform_conv():
+    """DCNv4-P4 inputs with a 512 -> 512 dense weight per kernel point."""
+    shape, inp = si.workload_core("dcnv4_p4")
+    inp.update(si.deform_conv_weights(shape.K, shape.G * shape.C, 512, shape.dtype, 9))
+    return shape, inp
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -583,7 +608,7 @@ def run_reference(args, world, rank):
 
 
 CASES = ("dcnv4_p4", "dcnv3_p3", "dcnv3_p3_dil2", "dcnv4_p4_bwd", "sparse4d", "sparse4d_bwd", "roi_pool",
-         "dcnv4_p4_proj")
+         "dcnv4_p4_proj", "dcnv2_p4_deform_conv")
 
 
 def run_case(name: str, calls: int) -> None:
@@ -614,10 +639,14 @@ def run_case(name: str, calls: int) -> None:
         t = [inp[k].to(dev) for k in ("x", "rois", "offset")]
         call = lambda: dcn.deform_roi_pool_forward(*t, pooled=(rs.PH, rs.PW), sampling=rs.S,
                                                    spatial_scale=rs.spatial_scale, gamma=rs.gamma)
-    else:
+    elif name == "dcnv4_p4_proj":
         shape, inp = si.workload_proj()
         t = [inp[k].to(dev) for k in ("x", "offset", "mask", "weight", "bias")]
         call = lambda: dcn.dcn_core_forward_proj(*t, group=shape.G)
+    else:
+        shape, inp = workload_deform_conv()
+        t = [inp[k].to(dev) for k in ("x", "offset", "mask", "weight", "bias")]
+        call = lambda: dcn.dcn_deform_conv_forward(*t, group=shape.G)
     for _ in range(calls):
         call()
     torch.cuda.synchronize()

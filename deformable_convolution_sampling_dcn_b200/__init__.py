@@ -4,6 +4,7 @@ Thin Python front end of libdcn_b200.so (C ABI in include/dcn_b200.h):
 
     dcn_core_forward / dcn_core_backward     DCNv2/v3/v4 sampling core
     dcn_core_forward_proj                    the core fused with its 1x1 projection (DCNv4 module)
+    dcn_deform_conv_forward                  modulated deformable convolution, weight per point (DCNv2)
     deform_agg_forward / deform_agg_backward Sparse4D multi-camera aggregation
     deform_roi_pool_forward                  deformable RoI pooling
     DCNCoreFunction, DeformAggFunction       autograd wrappers over the above
@@ -20,10 +21,11 @@ import torch
 
 from ._binding import (ABI_VERSION, EXPORTS, DaggParams, DcnError, DcnParams, DroiParams, core_params,
                        dcn_core_backward, dcn_core_forward, dcn_core_forward_proj, dcn_core_output_hw,
+                       dcn_deform_conv_forward,
                        deform_agg_backward,
                        deform_agg_forward, deform_roi_pool_forward, lib)
 
-__all__ = ["dcn_core_forward", "dcn_core_forward_proj", "dcn_core_backward", "dcn_core_output_hw", "deform_agg_forward",
+__all__ = ["dcn_core_forward", "dcn_core_forward_proj", "dcn_deform_conv_forward", "dcn_core_backward", "dcn_core_output_hw", "deform_agg_forward",
            "deform_agg_backward", "deform_roi_pool_forward", "DroiParams", "DCNCoreFunction", "DeformAggFunction", "shard_range", "lib", "DcnError",
            "DcnParams", "DaggParams", "core_params", "EXPORTS", "ABI_VERSION"]
 

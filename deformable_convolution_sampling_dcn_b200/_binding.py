@@ -27,7 +27,7 @@ _DTYPE_CODE = {torch.float32: DCN_F32, torch.float16: DCN_F16, torch.bfloat16: D
 EXPORTS = ("dcn_core_output_hw", "dcn_core_forward", "dcn_core_backward", "deform_agg_forward",
            "deform_agg_backward", "dcn_status_string", "dcn_last_error_detail", "dcn_abi_version",
            "dcn_take_device_error", "deform_roi_pool_forward", "dcn_core_forward_proj",
-           "dcn_selftest_bounded_wait")
+           "dcn_selftest_bounded_wait", "dcn_deform_conv_forward")
 ABI_VERSION = 1
 
 
@@ -81,6 +81,8 @@ def _declare(lib):
     lib.deform_roi_pool_forward.restype = st
     lib.dcn_core_forward_proj.argtypes = [P, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp]
     lib.dcn_core_forward_proj.restype = st
+    lib.dcn_deform_conv_forward.argtypes = [P, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp]
+    lib.dcn_deform_conv_forward.restype = st
     lib.dcn_selftest_bounded_wait.argtypes = [ctypes.c_int32, vp]
     lib.dcn_selftest_bounded_wait.restype = st
     lib.dcn_take_device_error.argtypes = []
@@ -221,6 +223,42 @@ def dcn_core_forward_proj(x: torch.Tensor, offset: torch.Tensor, mask: torch.Ten
     check(lib().dcn_core_forward_proj(ctypes.byref(p), cout, x.data_ptr(), offset.data_ptr(), mask.data_ptr(),
                                       weight.data_ptr(), None if bias is None else bias.data_ptr(),
                                       out.data_ptr(), _stream(x)))
+    return out
+
+
+def dcn_deform_conv_forward(x: torch.Tensor, offset: torch.Tensor, mask: torch.Tensor, weight: torch.Tensor,
+                            bias: Optional[torch.Tensor] = None, *, group: int, kernel=(3, 3), stride=(1, 1),
+                            pad=(1, 1), dil=(1, 1), offset_scale: float = 1.0, softmax: bool = False,
+                            out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out [B,Ho,Wo,Cout] = bias + sum_k weight[:, k, :] . (m_k x(p_k)): modulated deformable convolution
+    with weight [Cout, K, G*C] in one kernel; see dcn_b200.h."""
+    _cuda_tensor("x", x)
+    p = core_params(x, group, kernel, stride, pad, dil, offset_scale, softmax)
+    Ho, Wo = dcn_core_output_hw(p)
+    K = p.kh * p.kw
+    _cuda_tensor("offset", offset, x.dtype)
+    _cuda_tensor("mask", mask, x.dtype)
+    _cuda_tensor("weight", weight, x.dtype)
+    if tuple(offset.shape) != (p.B, Ho, Wo, p.G, K, 2):
+        raise ValueError(f"offset shape {tuple(offset.shape)} != {(p.B, Ho, Wo, p.G, K, 2)}")
+    if tuple(mask.shape) != (p.B, Ho, Wo, p.G, K):
+        raise ValueError(f"mask shape {tuple(mask.shape)} != {(p.B, Ho, Wo, p.G, K)}")
+    if weight.dim() != 3 or tuple(weight.shape[1:]) != (K, p.G * p.C):
+        raise ValueError(f"weight shape {tuple(weight.shape)} != (Cout, {K}, {p.G * p.C})")
+    cout = int(weight.shape[0])
+    if bias is not None:
+        _cuda_tensor("bias", bias, x.dtype)
+        if tuple(bias.shape) != (cout,):
+            raise ValueError(f"bias shape {tuple(bias.shape)} != ({cout},)")
+    if out is None:
+        out = torch.empty((p.B, Ho, Wo, cout), dtype=x.dtype, device=x.device)
+    else:
+        _cuda_tensor("out", out, x.dtype)
+        if tuple(out.shape) != (p.B, Ho, Wo, cout):
+            raise ValueError("out has the wrong shape")
+    check(lib().dcn_deform_conv_forward(ctypes.byref(p), cout, x.data_ptr(), offset.data_ptr(), mask.data_ptr(),
+                                        weight.data_ptr(), None if bias is None else bias.data_ptr(),
+                                        out.data_ptr(), _stream(x)))
     return out
 
 

@@ -162,24 +162,26 @@ dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offs
     return cuda_status(e, "dcn_core_forward launch");
 }
 
-dcn_status dcn_core_forward_proj(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
-                                 const void *mask, const void *weight, const void *bias, void *out,
-                                 dcn_stream_t stream) {
+namespace {
+
+dcn_status proj_call(const dcn_params *p, int32_t Cout, const void *x, const void *offset, const void *mask,
+                     const void *weight, const void *bias, void *out, dcn_stream_t stream, bool per_point,
+                     const char *what) {
     int Ho, Wo;
     dcn_status s = check_core(p, &Ho, &Wo);
     if (s != DCN_OK) return s;
     if (p->dtype != DCN_F16 && p->dtype != DCN_BF16)
-        return fail(DCN_ERR_UNSUPPORTED, "the fused projection takes fp16 or bf16 (dtype %d)", p->dtype);
-    if (p->C > 64) return fail(DCN_ERR_UNSUPPORTED, "the fused projection takes C <= 64 (C = %d)", p->C);
+        return fail(DCN_ERR_UNSUPPORTED, "the fused contraction takes fp16 or bf16 (dtype %d)", p->dtype);
+    if (p->C > 64) return fail(DCN_ERR_UNSUPPORTED, "the fused contraction takes C <= 64 (C = %d)", p->C);
     const long long GC = (long long)p->G * p->C;
     if (GC % 64 != 0 || GC > 512)
-        return fail(DCN_ERR_UNSUPPORTED, "the fused projection takes G*C in {64, 128, ..., 512} (G*C = %lld)", GC);
+        return fail(DCN_ERR_UNSUPPORTED, "the fused contraction takes G*C in {64, 128, ..., 512} (G*C = %lld)", GC);
     if ((long long)p->kh * p->kw > 25)
-        return fail(DCN_ERR_UNSUPPORTED, "the fused projection takes kh*kw <= 25");
+        return fail(DCN_ERR_UNSUPPORTED, "the fused contraction takes kh*kw <= 25");
     if (Cout < 8 || Cout > 512 || Cout % 8 != 0)
         return fail(DCN_ERR_UNSUPPORTED, "Cout must be a multiple of 8 in [8, 512] (Cout = %d)", Cout);
     if ((long long)p->H * p->W >= (1LL << 31) || (long long)p->B * Ho * Wo >= (1LL << 31))
-        return fail(DCN_ERR_UNSUPPORTED, "the fused projection takes H*W and B*Ho*Wo below 2^31");
+        return fail(DCN_ERR_UNSUPPORTED, "the fused contraction takes H*W and B*Ho*Wo below 2^31");
     if (p->B == 0) return DCN_OK;
     if (!x || !offset || !mask || !weight || !out)
         return fail(DCN_ERR_NULL, "x, offset, mask, weight and out are required");
@@ -193,7 +195,22 @@ dcn_status dcn_core_forward_proj(const dcn_params *p, int32_t Cout, const void *
     a.weight = weight;
     a.bias = bias;
     a.Cout = Cout;
-    return cuda_status(dcnb::launch_core_forward_proj(a, (cudaStream_t)stream), "dcn_core_forward_proj launch");
+    a.per_point = per_point;
+    return cuda_status(dcnb::launch_core_forward_proj(a, (cudaStream_t)stream), what);
+}
+
+}  // namespace
+
+dcn_status dcn_core_forward_proj(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
+                                 const void *mask, const void *weight, const void *bias, void *out,
+                                 dcn_stream_t stream) {
+    return proj_call(p, Cout, x, offset, mask, weight, bias, out, stream, false, "dcn_core_forward_proj launch");
+}
+
+dcn_status dcn_deform_conv_forward(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
+                                   const void *mask, const void *weight, const void *bias, void *out,
+                                   dcn_stream_t stream) {
+    return proj_call(p, Cout, x, offset, mask, weight, bias, out, stream, true, "dcn_deform_conv_forward launch");
 }
 
 dcn_status dcn_core_backward(const dcn_params *p, const void *x, const void *offset, const void *mask,

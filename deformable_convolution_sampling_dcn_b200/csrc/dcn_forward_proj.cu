@@ -4,6 +4,13 @@
 //     out[p, o] = bias[o] + sum_j Wt[o, j] * core[p, j],  j = g*C + c.
 // The core tile never leaves the SM.
 //
+// The same kernel runs the modulated deformable convolution (DCNv2 page,
+// section 1: every kernel point has its own dense weight):
+//     out[p, o] = bias[o] + sum_k sum_j Wt[o, k, j] * m_k * x_j(p + p_k + dp_k).
+// There the K-blocks run over (kernel point, 64 channels) and each item
+// samples only its K-block's point, so the tensor core contracts over all
+// K * G * C sampled values instead of the G * C core values.
+//
 // Work split.  The B*Ho*Wo pixels are cut into one contiguous range per CTA
 // (persistent grid, one CTA per SM), processed in chunks of at most 128
 // pixels.  Per chunk:
@@ -54,7 +61,9 @@ struct ProjParams {
     long long P;        // output pixels B*Ho*Wo
     int Cout;
     int MB;             // ceil(Cout / 128) output-channel blocks
-    int KB;             // G*C / 64 channel blocks
+    int KB;             // 64-channel K-blocks of the contraction
+    int cbk;            // K-blocks per kernel point (KB when the points are summed first)
+    int per_point;      // 1: deformable convolution, one K-block per (point, channel block)
     int n_cta;
     int npad_max;       // largest padded chunk of any CTA (B operand rows)
     int tmem_cols;      // allocated tensor-memory columns (power of two >= 32)
@@ -72,15 +81,16 @@ __device__ __align__(16) unsigned char g_zero_row[128];
 // list is dealt to the gather warps in steps of IPW items, round-robin, so
 // every warp gets the same number of steps whatever the K-block sizes.
 struct ItemPos {
-    int kb, g, px;
+    int kb, k, g, px;  // K-block, kernel point (per-point mode), group, pixel in the chunk
 };
-__device__ __forceinline__ ItemPos item_pos(int item, int n_px, int per_kb, int gpb) {
+__device__ __forceinline__ ItemPos item_pos(int item, int n_px, int per_kb, int gpb, int cbk) {
     ItemPos r;
     r.kb = item / per_kb;
     const int j = item - r.kb * per_kb;
     const int gl = j / n_px;
     r.px = j - gl * n_px;
-    r.g = r.kb * gpb + gl;
+    r.k = r.kb / cbk;
+    r.g = (r.kb - r.k * cbk) * gpb + gl;
     return r;
 }
 
@@ -92,7 +102,7 @@ __device__ __forceinline__ void load_raw(const ProjParams &p, long long c0, int 
     const CoreArgs &a = p.a;
     const int K = a.kh * a.kw;
     const bool valid = item < total;
-    const ItemPos ip = item_pos(valid ? item : 0, n_px, per_kb, 64 / a.C);
+    const ItemPos ip = item_pos(valid ? item : 0, n_px, per_kb, 64 / a.C, p.cbk);
     const long long mi = (c0 + ip.px) * a.G + ip.g;
     const T *off = static_cast<const T *>(a.offset);
     const T *msk = static_cast<const T *>(a.mask);
@@ -136,7 +146,7 @@ __device__ __forceinline__ void gather_step(const ProjParams &p, int ci, long lo
     const int gi = lane / LPI, q = lane % LPI;  // gather role
     const int item = base + gi;
     const bool valid = item < total;
-    const ItemPos ip = item_pos(valid ? item : 0, n_px, per_kb, gpb);
+    const ItemPos ip = item_pos(valid ? item : 0, n_px, per_kb, gpb, p.cbk);
     const unsigned pix = (unsigned)(c0 + ip.px);
     const unsigned b = pix / HoWo;
     const T *xb = xg + (long long)b * a.H * a.W * GC + ip.g * a.C + q * V;
@@ -148,7 +158,7 @@ __device__ __forceinline__ void gather_step(const ProjParams &p, int ci, long lo
         const int ri = lane % IPW, k0 = lane / IPW;
         const int item_r = base + ri;
         const bool valid_r = item_r < total;
-        const ItemPos ipr = item_pos(valid_r ? item_r : 0, n_px, per_kb, gpb);
+        const ItemPos ipr = item_pos(valid_r ? item_r : 0, n_px, per_kb, gpb, p.cbk);
         const unsigned rem = (unsigned)(c0 + ipr.px) % HoWo;
         const int ho = (int)(rem / (unsigned)a.Wo), wo = (int)(rem % (unsigned)a.Wo);
         float m[NT];
@@ -240,9 +250,10 @@ __device__ __forceinline__ void gather_step(const ProjParams &p, int ci, long lo
             inv_sum = 1.0f / sum;
         }
         bool nan_pos = false;
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k) {
-            if (k >= K) break;
+        // all K points summed (core + projection), or only this K-block's point
+        // (deformable convolution: the points are contracted by the weight)
+        const int k_lo = p.per_point ? ip.k : 0, k_hi = p.per_point ? ip.k + 1 : K;
+        for (int k = k_lo; k < k_hi; ++k) {
             const int2 kt = ktab[k];
             const float2 d = load_pair(o_item + 2 * k);
             float m = load_scalar(m_item + k);
@@ -548,6 +559,12 @@ template <typename T, int LPI>
 cudaError_t launch_lpi(const CUtensorMap &map, const ProjParams &p, size_t min_smem, cudaStream_t stream) {
     const int K = p.a.kh * p.a.kw;
     auto pick = [&](size_t need) { return need > min_smem ? need : min_smem; };
+    if (p.per_point) {
+        // one tap per item: every lane computes its own
+        const size_t smem = pick(proj_smem(p.npad_max, LPI, 25, false));
+        return p.a.softmax ? launch_one<T, LPI, true, 25, false>(map, p, smem, stream)
+                           : launch_one<T, LPI, false, 25, false>(map, p, smem, stream);
+    }
     if (K <= 9) {
         // records for 2..8 lanes per item; a single-lane item computes its own taps
         constexpr bool R = LPI >= 2;
@@ -572,7 +589,10 @@ cudaError_t launch_t(const ProjArgs &pa, cudaStream_t stream) {
     p.P = (long long)a.B * a.Ho * a.Wo;
     p.Cout = pa.Cout;
     p.MB = (pa.Cout + 127) / 128;
-    p.KB = a.G * a.C / 64;
+    const int K = a.kh * a.kw;
+    p.per_point = pa.per_point ? 1 : 0;
+    p.cbk = a.G * a.C / 64;
+    p.KB = pa.per_point ? K * p.cbk : p.cbk;
     p.err = dev->err;
     long long n_cta = dev->sms;
     if (n_cta * 16 > p.P) n_cta = (p.P + 15) / 16;  // at least 16 pixels per CTA
@@ -592,7 +612,8 @@ cudaError_t launch_t(const ProjArgs &pa, cudaStream_t stream) {
     if (proj_smem(p.npad_max, 2, 9, true) > (size_t)dev->smem_optin) return cudaErrorInvalidConfiguration;
 
     CUtensorMap map;
-    const cuuint64_t dims[2] = {(cuuint64_t)a.G * a.C, (cuuint64_t)pa.Cout};
+    // weight [Cout, G*C] (projection) or [Cout, K, G*C] (deformable convolution)
+    const cuuint64_t dims[2] = {(cuuint64_t)(pa.per_point ? K : 1) * a.G * a.C, (cuuint64_t)pa.Cout};
     const cuuint64_t strides[1] = {dims[0] * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)p.w_box_rows};
     const cuuint32_t estr[2] = {1, 1};

@@ -30,9 +30,10 @@ struct CoreArgs {
 // Forward core followed by its pointwise projection (fp16/bf16 only).
 struct ProjArgs {
     CoreArgs core;       // core.out is the projected output [B, Ho, Wo, Cout]
-    const void *weight;  // [Cout, G*C]
+    const void *weight;  // [Cout, G*C], or [Cout, K, G*C] when per_point
     const void *bias;    // [Cout] or nullptr
     int Cout;
+    bool per_point;      // deformable convolution: a dense weight per kernel point
 };
 
 struct AggArgs {

@@ -14,8 +14,9 @@
  * points of the (pixel, group) as in DCNv3 or used raw as in DCNv4 (YOLOv11 +
  * DCNv4 article, section 1.1), and the K samples are summed in fp32.  The
  * pointwise projection that follows the core in the DCNv4 module (1x1
- * convolution with bias) is available fused with it (dcn_core_forward_proj);
- * the dense per-point weight w(pn) of DCNv1/v2 is not part of this library.
+ * convolution with bias) is available fused with it (dcn_core_forward_proj),
+ * and so is the dense per-point weight w(pn) of DCNv1/v2 (the modulated
+ * deformable convolution, dcn_deform_conv_forward).
  *
  * Conventions shared by every call:
  *   - All tensor pointers are DEVICE pointers to dense, C-contiguous buffers
@@ -129,6 +130,28 @@ dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offs
 dcn_status dcn_core_forward_proj(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
                                  const void *mask, const void *weight, const void *bias, void *out,
                                  dcn_stream_t stream);
+
+/*
+ * Modulated deformable convolution with a dense weight per kernel point (the
+ * DCNv2 page "DCNv2实战：在YOLOv5中替换普通卷积...", section 1:
+ * y(p0) = sum_n w(pn) * x(p0 + pn + dpn) * dm_n; with unit masks it is the DCNv1
+ * page's section-1 formula), in one kernel:
+ *   out[b, ho, wo, o] = bias[o] + sum_k sum_j weight[o, k, j] * m_k * x_j(p_k),
+ *   j = g*C + c; offset and modulation of point k shared by deformable group g.
+ *   weight [Cout, K, G*C]     storage dtype (a Conv2d weight [Cout, G*C, kh, kw]
+ *                             permuted to point-major)
+ *   bias   [Cout]             storage dtype, or NULL
+ *   out    [B, Ho, Wo, Cout]  storage dtype
+ * x, offset and mask are as for dcn_core_forward (softmax mode normalises the
+ * K masks of each (pixel, group) first).  Each sampled, modulated value is
+ * formed in fp32 and rounded once to the storage dtype as the tensor-core
+ * operand; the contraction over the K*G*C values accumulates in fp32.  The
+ * K*G*C-wide column matrix never reaches device memory.  Same support,
+ * alignment and error rules as dcn_core_forward_proj.
+ */
+dcn_status dcn_deform_conv_forward(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
+                                   const void *mask, const void *weight, const void *bias, void *out,
+                                   dcn_stream_t stream);
 
 /*
  * Backward core: gradients of L = <grad_out, out> with respect to x, offset

@@ -320,3 +320,12 @@ def workload_proj() -> Tuple[CoreShape, Dict[str, torch.Tensor]]:
     shape, inp = workload_core("dcnv4_p4")
     inp.update(proj_inputs(shape.G * shape.C, PROJ_COUT_P4, shape.dtype, SEEDS["dcnv4_p4_proj"]))
     return shape, inp
+
+
+def deform_conv_weights(K: int, cin: int, cout: int, dtype: str, seed: int) -> Dict[str, torch.Tensor]:
+    """weight [cout, K, cin] ~ N(0, 1/(K*cin)) (a Conv2d weight permuted to
+    point-major) and bias [cout] ~ N(0, 0.1^2), rounded once to the storage dtype."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    w = rng.standard_normal((cout, K, cin)) / np.sqrt(K * cin)
+    b = rng.standard_normal(cout) * 0.1
+    return {"weight": _round(w, dtype), "bias": _round(b, dtype)}

@@ -170,3 +170,12 @@ def test_proj_checks(lib):
 def test_selftest_limit_checked_on_host(lib):
     assert lib.dcn_selftest_bounded_wait(0, None) == B.DCN_ERR_SHAPE
     assert lib.dcn_selftest_bounded_wait(20_000_000, None) == B.DCN_ERR_SHAPE
+
+
+def test_deform_conv_checks(lib):
+    p = params(G=16, C=32)
+    f = lib.dcn_deform_conv_forward
+    assert f(ctypes.byref(p), 256, 16, 16, 16, 0, None, 16, None) == B.DCN_ERR_NULL
+    assert f(ctypes.byref(p), 100, 16, 16, 16, 16, None, 16, None) == B.DCN_ERR_UNSUPPORTED
+    assert f(ctypes.byref(params(G=16, C=32, dtype=0)), 64, 16, 16, 16, 16, None, 16, None) == B.DCN_ERR_UNSUPPORTED
+    assert f(ctypes.byref(params(B=0, G=16, C=32)), 64, None, None, None, None, None, None, None) == B.DCN_OK

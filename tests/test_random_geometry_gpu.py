@@ -130,3 +130,41 @@ def test_roi_pool(i, cuda_dev):
     out = d.deform_roi_pool_forward(*(inp[k].to(cuda_dev) for k in ("x", "rois", "offset")), **kw)
     torch.cuda.synchronize()
     assert_close_fwd(out, oracle.roi_pool_forward(inp["x"], inp["rois"], inp["offset"], **kw), f"random roi {i}")
+
+
+def draw_agg(i):
+    r = np.random.default_rng(11000 + i)
+    dt = ["f32", "f16", "bf16"][r.integers(3)]
+    es = 4 if dt == "f32" else 2
+    C = int(r.choice([c for c in (4, 8, 16, 32, 64) if (c * es) % 16 == 0]))
+    G = int(r.choice([1, 2, 4, 8, 16]))
+    if i % 2 == 0:  # every other case takes a 512/1024/2048-byte row (the all-groups kernels)
+        row = int(r.choice([512, 1024, 2048]))
+        G = max(1, row // (C * es))
+        C = row // (G * es)
+    cams = int(r.integers(1, 7))
+    scales = tuple((int(r.integers(1, 20)), int(r.integers(1, 30))) for _ in range(int(r.integers(1, 5))))
+    shape = si.AggShape(B=int(r.integers(1, 3)), num_cams=cams, scales=scales, num_anchors=int(r.integers(1, 60)),
+                        num_pts=int(r.integers(1, 14)), G=G, C=C, dtype=dt)
+    lo, hi = [(0.0, 1.0), (-0.1, 1.1), (-0.5, 1.5)][r.integers(3)]
+    return shape, lo, hi
+
+
+AGG_KEYS = ("feat", "spatial_shape", "scale_start_index", "sampling_location", "weights")
+
+
+@pytest.mark.parametrize("i", range(16))
+def test_aggregation(i, cuda_dev):
+    import deformable_convolution_sampling_dcn_b200 as d
+
+    shape, lo, hi = draw_agg(i)
+    inp = si.agg_inputs(shape, 12000 + i, with_grad_out=True, loc_lo=lo, loc_hi=hi)
+    t = [inp[k].to(cuda_dev) for k in AGG_KEYS]
+    out = d.deform_agg_forward(*t)
+    gf, gl, gw = d.deform_agg_backward(*t, inp["grad_out"].to(cuda_dev))
+    torch.cuda.synchronize()
+    assert_close_fwd(out, oracle.agg_forward(*(inp[k] for k in AGG_KEYS)), f"random agg forward {i}")
+    ref = oracle.agg_backward(*(inp[k] for k in AGG_KEYS), inp["grad_out"])
+    assert_close_bwd(gf, ref["grad_feat"], f"random agg grad_feat {i}")
+    assert_close_bwd(gl, ref["grad_loc"], f"random agg grad_loc {i}")
+    assert_close_bwd(gw, ref["grad_weights"], f"random agg grad_weights {i}")
