@@ -55,6 +55,26 @@ constexpr int kMaxChunk = 128;          // pixels per chunk (MMA N <= 128)
 constexpr int kBSlots = 4;             // B-operand ring: K-blocks in flight
 constexpr uint64_t kProjWaitNs = 1000000000ull;
 
+// Unsigned division by a divisor fixed for a launch or a chunk, without the
+// hardware division sequence: q = mulhi(n, m) with m = floor((2^32 - 1) / d)
+// underestimates n / d by at most one for n < 2^31 (n*m/2^32 lies in
+// (n/d - 1, n/d)), so one remainder check makes it exact (the round-down
+// reciprocal method of Granlund and Montgomery, "Division by invariant
+// integers using multiplication", 1994).
+struct FastDiv {
+    unsigned d, m;
+};
+__host__ __device__ inline FastDiv make_fastdiv(unsigned d) { return FastDiv{d, 0xFFFFFFFFu / d}; }
+__device__ __forceinline__ unsigned fdiv(unsigned n, FastDiv f, unsigned &r) {
+    unsigned q = __umulhi(n, f.m);
+    r = n - q * f.d;
+    if (r >= f.d) {
+        ++q;
+        r -= f.d;
+    }
+    return q;
+}
+
 struct ProjParams {
     CoreArgs a;
     const void *bias;   // [Cout] storage type, or nullptr
@@ -64,6 +84,8 @@ struct ProjParams {
     int KB;             // 64-channel K-blocks of the contraction
     int cbk;            // K-blocks per kernel point (KB when the points are summed first)
     int per_point;      // 1: deformable convolution, one K-block per (point, channel block)
+    int lg_gpb;         // log2 of the groups per K-block (64 / C)
+    FastDiv fd_cbk, fd_howo, fd_wo;  // K-blocks per point, Ho*Wo, Wo
     int n_cta;
     int npad_max;       // largest padded chunk of any CTA (B operand rows)
     int tmem_cols;      // allocated tensor-memory columns (power of two >= 32)
@@ -83,26 +105,28 @@ __device__ __align__(16) unsigned char g_zero_row[128];
 struct ItemPos {
     int kb, k, g, px;  // K-block, kernel point (per-point mode), group, pixel in the chunk
 };
-__device__ __forceinline__ ItemPos item_pos(int item, int n_px, int per_kb, int gpb, int cbk) {
+__device__ __forceinline__ ItemPos item_pos(int item, FastDiv fd_npx, const ProjParams &p) {
+    // item = (kb * gpb + gl) * n_px + px, kb = k * cbk + cb, g = cb * gpb + gl
     ItemPos r;
-    r.kb = item / per_kb;
-    const int j = item - r.kb * per_kb;
-    const int gl = j / n_px;
-    r.px = j - gl * n_px;
-    r.k = r.kb / cbk;
-    r.g = (r.kb - r.k * cbk) * gpb + gl;
+    unsigned px, cb;
+    const unsigned q = fdiv((unsigned)item, fd_npx, px);
+    r.px = (int)px;
+    r.kb = (int)(q >> p.lg_gpb);
+    const int gl = (int)(q & ((1u << p.lg_gpb) - 1u));
+    r.k = (int)fdiv((unsigned)r.kb, p.fd_cbk, cb);
+    r.g = ((int)cb << p.lg_gpb) + gl;
     return r;
 }
 
 // Offsets and masks of points k0, k0 + LPI, ... of flat item `item` (the
 // record role's raw taps), loaded one step ahead of their use.
 template <typename T, int LPI, bool SOFTMAX, int NT>
-__device__ __forceinline__ void load_raw(const ProjParams &p, long long c0, int n_px, int per_kb, int total,
+__device__ __forceinline__ void load_raw(const ProjParams &p, long long c0, FastDiv fd_npx, int total,
                                          int item, int k0, float *dx, float *dy, float *m) {
     const CoreArgs &a = p.a;
     const int K = a.kh * a.kw;
     const bool valid = item < total;
-    const ItemPos ip = item_pos(valid ? item : 0, n_px, per_kb, 64 / a.C, p.cbk);
+    const ItemPos ip = item_pos(valid ? item : 0, fd_npx, p);
     const long long mi = (c0 + ip.px) * a.G + ip.g;
     const T *off = static_cast<const T *>(a.offset);
     const T *msk = static_cast<const T *>(a.mask);
@@ -131,8 +155,8 @@ __device__ __forceinline__ void load_raw(const ProjParams &p, long long c0, int 
 // records and gather their 16-byte channel chunks of the four corners
 // through L1.  Otherwise every lane of an item computes the taps itself.
 template <typename T, int LPI, bool SOFTMAX, int KMAX, bool RECORDS, int NT>
-__device__ __forceinline__ void gather_step(const ProjParams &p, int ci, long long c0, int n_px, int per_kb,
-                                            int total, int base, int lane, unsigned char *bring, int slot_bytes,
+__device__ __forceinline__ void gather_step(const ProjParams &p, int ci, long long c0, FastDiv fd_npx, int total,
+                                            int base, int lane, unsigned char *bring, int slot_bytes,
                                             float4 *rec_w, int4 *rec_o, const int2 *ktab, const float *dx,
                                             const float *dy, const float *m_raw) {
     constexpr int V = Storage<T>::kVec;
@@ -140,15 +164,14 @@ __device__ __forceinline__ void gather_step(const ProjParams &p, int ci, long lo
     const CoreArgs &a = p.a;
     const int K = a.kh * a.kw;
     const int GC = a.G * a.C;
-    const int gpb = 64 / a.C;
-    const unsigned HoWo = (unsigned)a.Ho * (unsigned)a.Wo;
     const T *__restrict__ xg = static_cast<const T *>(a.x);
     const int gi = lane / LPI, q = lane % LPI;  // gather role
     const int item = base + gi;
     const bool valid = item < total;
-    const ItemPos ip = item_pos(valid ? item : 0, n_px, per_kb, gpb, p.cbk);
+    const ItemPos ip = item_pos(valid ? item : 0, fd_npx, p);
     const unsigned pix = (unsigned)(c0 + ip.px);
-    const unsigned b = pix / HoWo;
+    unsigned rem;
+    const unsigned b = fdiv(pix, p.fd_howo, rem);
     const T *xb = xg + (long long)b * a.H * a.W * GC + ip.g * a.C + q * V;
     float acc[V];
 #pragma unroll
@@ -158,9 +181,10 @@ __device__ __forceinline__ void gather_step(const ProjParams &p, int ci, long lo
         const int ri = lane % IPW, k0 = lane / IPW;
         const int item_r = base + ri;
         const bool valid_r = item_r < total;
-        const ItemPos ipr = item_pos(valid_r ? item_r : 0, n_px, per_kb, gpb, p.cbk);
-        const unsigned rem = (unsigned)(c0 + ipr.px) % HoWo;
-        const int ho = (int)(rem / (unsigned)a.Wo), wo = (int)(rem % (unsigned)a.Wo);
+        const ItemPos ipr = item_pos(valid_r ? item_r : 0, fd_npx, p);
+        unsigned rem_r, wo_r;
+        fdiv((unsigned)(c0 + ipr.px), p.fd_howo, rem_r);
+        const int ho = (int)fdiv(rem_r, p.fd_wo, wo_r), wo = (int)wo_r;
         float m[NT];
 #pragma unroll
         for (int j = 0; j < NT; ++j) m[j] = m_raw[j];
@@ -236,8 +260,8 @@ __device__ __forceinline__ void gather_step(const ProjParams &p, int ci, long lo
         }
     } else if (valid) {
         // ---- every lane computes the taps of its item
-        const unsigned rem = pix % HoWo;
-        const int ho = (int)(rem / (unsigned)a.Wo), wo = (int)(rem % (unsigned)a.Wo);
+        unsigned wo_u;
+        const int ho = (int)fdiv(rem, p.fd_wo, wo_u), wo = (int)wo_u;
         const long long mi = (long long)pix * a.G + ip.g;
         const T *o_item = static_cast<const T *>(a.offset) + mi * K * 2;
         const T *m_item = static_cast<const T *>(a.mask) + mi * K;
@@ -441,8 +465,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             chunk_range(r0, r1, ci, n_chunks, c0, c1);
             const int n_px = (int)(c1 - c0);
             const int npad = (n_px + 15) & ~15;
-            const int per_kb = n_px * (64 / a.C);
+            const int per_kb = n_px << p.lg_gpb;
             const int total = per_kb * p.KB;
+            const FastDiv fd_npx = make_fastdiv((unsigned)n_px), fd_pkb = make_fastdiv((unsigned)per_kb);
+            unsigned fr;
             const int n_steps = (total + IPW - 1) / IPW;
             int waited = -1;    // slots of K-blocks <= waited are known to be free
             int signaled = 0;   // K-blocks < signaled are handed to the tensor core by this warp
@@ -471,7 +497,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 return true;
             };
             float dx[NT], dy[NT], m[NT];
-            if (RECORDS) load_raw<T, LPI, SOFTMAX, NT>(p, c0, n_px, per_kb, total, warp * IPW + ri, k0, dx, dy, m);
+            if (RECORDS) load_raw<T, LPI, SOFTMAX, NT>(p, c0, fd_npx, total, warp * IPW + ri, k0, dx, dy, m);
             for (int st = warp; st < n_steps; st += kGatherWarps) {
                 const int first = st * IPW;
                 const int last = (first + IPW < total ? first + IPW : total) - 1;
@@ -479,7 +505,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 // warp: hand them over before waiting for any slot, so that every
                 // wait below depends only on K-blocks this warp has already
                 // handed over (a step spans at most four K-blocks, the ring size)
-                if (!signal(first / per_kb) || !slot_free(last / per_kb)) {
+                if (!signal((int)fdiv((unsigned)first, fd_pkb, fr)) ||
+                    !slot_free((int)fdiv((unsigned)last, fd_pkb, fr))) {
                     stop = true;
                     break;
                 }
@@ -492,11 +519,11 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 }
                 const int nxt = st + kGatherWarps;
                 if (RECORDS && nxt < n_steps)
-                    load_raw<T, LPI, SOFTMAX, NT>(p, c0, n_px, per_kb, total, nxt * IPW + ri, k0, dx, dy, m);
-                gather_step<T, LPI, SOFTMAX, KMAX, RECORDS, NT>(p, ci, c0, n_px, per_kb, total, first, lane, bring,
+                    load_raw<T, LPI, SOFTMAX, NT>(p, c0, fd_npx, total, nxt * IPW + ri, k0, dx, dy, m);
+                gather_step<T, LPI, SOFTMAX, KMAX, RECORDS, NT>(p, ci, c0, fd_npx, total, first, lane, bring,
                                                                  slot_bytes, rec_w, rec_o, ktab, cdx, cdy, cm);
                 // every K-block before the one this warp's next step starts in is done
-                if (!signal(nxt < n_steps ? (nxt * IPW) / per_kb : p.KB)) {
+                if (!signal(nxt < n_steps ? (int)fdiv((unsigned)(nxt * IPW), fd_pkb, fr) : p.KB)) {
                     stop = true;
                     break;
                 }
@@ -593,6 +620,11 @@ cudaError_t launch_t(const ProjArgs &pa, cudaStream_t stream) {
     p.per_point = pa.per_point ? 1 : 0;
     p.cbk = a.G * a.C / 64;
     p.KB = pa.per_point ? K * p.cbk : p.cbk;
+    p.lg_gpb = 0;
+    while ((a.C << p.lg_gpb) < 64) ++p.lg_gpb;
+    p.fd_cbk = make_fastdiv((unsigned)p.cbk);
+    p.fd_howo = make_fastdiv((unsigned)(a.Ho * a.Wo));
+    p.fd_wo = make_fastdiv((unsigned)a.Wo);
     p.err = dev->err;
     long long n_cta = dev->sms;
     if (n_cta * 16 > p.P) n_cta = (p.P + 15) / 16;  // at least 16 pixels per CTA
