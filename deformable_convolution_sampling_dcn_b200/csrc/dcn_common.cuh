@@ -23,6 +23,35 @@ template <> struct Storage<__nv_bfloat16> {
     static constexpr int kVec = 8;
 };
 
+// Unsigned division by a divisor fixed for a launch (or a chunk of work), without the
+// hardware division sequence: q = mulhi(n, m) with m = floor((2^32 - 1) / d)
+// underestimates n / d by at most one for n < 2^31 (n*m/2^32 lies in
+// (n/d - 1, n/d)), so one remainder check makes it exact (the round-down
+// reciprocal method of Granlund and Montgomery, "Division by invariant
+// integers using multiplication", 1994).
+struct FastDiv {
+    unsigned d, m;
+};
+__host__ __device__ inline FastDiv make_fastdiv(unsigned d) { return FastDiv{d, 0xFFFFFFFFu / d}; }
+__device__ __forceinline__ unsigned fdiv(unsigned n, FastDiv f, unsigned &r) {
+    unsigned q = __umulhi(n, f.m);
+    r = n - q * f.d;
+    if (r >= f.d) {
+        ++q;
+        r -= f.d;
+    }
+    return q;
+}
+
+// Divisors of a flat (b, ho, wo, g) item index (g fastest), for item indices
+// below 2^31.
+struct ItemDecode {
+    FastDiv g, wo, ho;
+};
+inline ItemDecode make_item_decode(int G, int Wo, int Ho) {
+    return ItemDecode{make_fastdiv((unsigned)G), make_fastdiv((unsigned)Wo), make_fastdiv((unsigned)Ho)};
+}
+
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__half v) { return __half2float(v); }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }

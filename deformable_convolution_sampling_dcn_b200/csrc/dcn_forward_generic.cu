@@ -17,7 +17,7 @@ namespace dcnb {
 namespace {
 
 template <typename T, int LPI, bool SOFTMAX>
-__global__ void __launch_bounds__(256) core_forward_generic(CoreArgs a) {
+__global__ void __launch_bounds__(256) core_forward_generic(CoreArgs a, ItemDecode dd) {
     constexpr int V = Storage<T>::kVec;
     constexpr int IPW = 32 / LPI;
     const int lane = threadIdx.x & 31;
@@ -35,14 +35,14 @@ __global__ void __launch_bounds__(256) core_forward_generic(CoreArgs a) {
     for (long long item = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * IPW + slot;
          item < n_items; item += warps_total * IPW) {
         int g, wo, ho, b;
-        if (n_items <= 0xffffffffLL) {  // 32-bit decode (the common case)
-            unsigned t = (unsigned)item;
-            g = (int)(t % (unsigned)a.G);
-            t /= (unsigned)a.G;
-            wo = (int)(t % (unsigned)a.Wo);
-            t /= (unsigned)a.Wo;
-            ho = (int)(t % (unsigned)a.Ho);
-            b = (int)(t / (unsigned)a.Ho);
+        if (n_items < (1LL << 31)) {  // 32-bit decode by multiply-high (the common case)
+            unsigned r;
+            unsigned t = fdiv((unsigned)item, dd.g, r);
+            g = (int)r;
+            t = fdiv(t, dd.wo, r);
+            wo = (int)r;
+            b = (int)fdiv(t, dd.ho, r);
+            ho = (int)r;
         } else {
             long long t = item;
             g = (int)(t % a.G);
@@ -121,10 +121,11 @@ cudaError_t launch_lpi(const CoreArgs &a, cudaStream_t stream) {
     const long long items_per_block = (threads / 32) * (32 / LPI);
     long long blocks = (n_items + items_per_block - 1) / items_per_block;
     if (blocks > 148LL * 64) blocks = 148LL * 64;  // grid-stride beyond this
+    const ItemDecode dd = make_item_decode(a.G, a.Wo, a.Ho);
     if (a.softmax)
-        core_forward_generic<T, LPI, true><<<(unsigned)blocks, threads, 0, stream>>>(a);
+        core_forward_generic<T, LPI, true><<<(unsigned)blocks, threads, 0, stream>>>(a, dd);
     else
-        core_forward_generic<T, LPI, false><<<(unsigned)blocks, threads, 0, stream>>>(a);
+        core_forward_generic<T, LPI, false><<<(unsigned)blocks, threads, 0, stream>>>(a, dd);
     return cudaGetLastError();
 }
 

@@ -64,6 +64,7 @@ cudaError_t launch_t(const CoreArgs &a, cudaStream_t stream, bool *handled) {
     if (RB != 32 && RB != 64 && RB != 128 && RB != 256) return cudaSuccess;
     const int K = a.kh * a.kw;
     if (K > 25 || a.W + 2 > 256) return cudaSuccess;
+    if ((long long)a.Ho * a.Wo >= (1LL << 31)) return cudaSuccess;  // plane index decode is 32-bit
     const int kmax = K <= 9 ? 9 : 25;
     auto enc = encode_fn();
     const DeviceInfo *dev = device_info();
@@ -76,6 +77,10 @@ cudaError_t launch_t(const CoreArgs &a, cudaStream_t stream, bool *handled) {
     s.row_bytes = (a.W + 2) * RB;
     s.box_rows = kBoxRows;
     s.err = dev->err;
+    s.fd_wo = make_fastdiv((unsigned)a.Wo);
+    s.fd_hw = make_fastdiv((unsigned)(a.Ho * a.Wo));
+    s.fd_g = make_fastdiv((unsigned)a.G);
+    s.fd_box = make_fastdiv((unsigned)kBoxRows);
     // One CTA of kStagedMaxThreads per SM: a producer warp stages the bands of
     // consecutive segments while the consumer warps gather.  Two band buffers
     // (the next segment loads while the current one is gathered) when they

@@ -55,26 +55,6 @@ constexpr int kMaxChunk = 128;          // pixels per chunk (MMA N <= 128)
 constexpr int kBSlots = 4;             // B-operand ring: K-blocks in flight
 constexpr uint64_t kProjWaitNs = 1000000000ull;
 
-// Unsigned division by a divisor fixed for a launch or a chunk, without the
-// hardware division sequence: q = mulhi(n, m) with m = floor((2^32 - 1) / d)
-// underestimates n / d by at most one for n < 2^31 (n*m/2^32 lies in
-// (n/d - 1, n/d)), so one remainder check makes it exact (the round-down
-// reciprocal method of Granlund and Montgomery, "Division by invariant
-// integers using multiplication", 1994).
-struct FastDiv {
-    unsigned d, m;
-};
-__host__ __device__ inline FastDiv make_fastdiv(unsigned d) { return FastDiv{d, 0xFFFFFFFFu / d}; }
-__device__ __forceinline__ unsigned fdiv(unsigned n, FastDiv f, unsigned &r) {
-    unsigned q = __umulhi(n, f.m);
-    r = n - q * f.d;
-    if (r >= f.d) {
-        ++q;
-        r -= f.d;
-    }
-    return q;
-}
-
 struct ProjParams {
     CoreArgs a;
     const void *bias;   // [Cout] storage type, or nullptr

@@ -60,6 +60,10 @@ struct StagedParams {
     unsigned int *err;  // device error word (bit 0: a TMA wait ran out)
     int threads;        // CTA size (multiple of 32, <= kStagedMaxThreads)
     int nbuf;           // band buffers (1 or 2): segment n uses buffer n % nbuf
+    FastDiv fd_wo;      // division by Wo
+    FastDiv fd_hw;      // division by Ho * Wo (used when n_items < 2^31)
+    FastDiv fd_g;       // division by G (used when n_items < 2^31)
+    FastDiv fd_box;     // division by box_rows
 };
 
 struct Segment {
@@ -71,23 +75,30 @@ __device__ __forceinline__ Segment make_segment(long long i0, long long iend, co
     const CoreArgs &a = s.a;
     Segment sg;
     const long long hw = (long long)a.Ho * a.Wo;
-    const long long plane = i0 / hw;
+    const bool small = s.n_items < (1LL << 31);  // 32-bit decode by multiply-high
+    unsigned r;
+    const long long plane = small ? (long long)fdiv((unsigned)i0, s.fd_hw, r) : i0 / hw;
     const int lp = (int)(i0 - plane * hw);
     sg.i0 = i0;
-    const int ho_a = lp / a.Wo;
+    const int ho_a = (int)fdiv((unsigned)lp, s.fd_wo, r);
     const long long lim = plane * hw + (long long)(ho_a + s.seg_rows) * a.Wo;
     const long long pend = (plane + 1) * hw;
     sg.i1 = iend < pend ? iend : pend;
     if (lim < sg.i1) sg.i1 = lim;
-    const int ho_b = (int)((sg.i1 - 1 - plane * hw) / a.Wo);
-    sg.b = (int)(plane / a.G);
-    sg.g = (int)(plane % a.G);
+    const int ho_b = (int)fdiv((unsigned)(sg.i1 - 1 - plane * hw), s.fd_wo, r);
+    if (small) {
+        sg.b = (int)fdiv((unsigned)plane, s.fd_g, r);
+        sg.g = (int)r;
+    } else {
+        sg.b = (int)(plane / a.G);
+        sg.g = (int)(plane % a.G);
+    }
     const int ys = ho_a * a.sh - a.ph - s.halo;
     const int ye = ho_b * a.sh - a.ph + (a.kh - 1) * a.dh + 1 + s.halo;
     sg.ys = ys < -1 ? -1 : ys;
     sg.ye = ye > a.H ? a.H : ye;
     // at least one box, so that column 0 of rows 0 and 1 always exists as zeros
-    sg.nbox = sg.ye >= sg.ys ? (sg.ye - sg.ys + s.box_rows) / s.box_rows : 1;
+    sg.nbox = sg.ye >= sg.ys ? (int)fdiv((unsigned)(sg.ye - sg.ys + s.box_rows), s.fd_box, r) : 1;
     return sg;
 }
 
@@ -230,8 +241,9 @@ __global__ void __launch_bounds__(kStagedMaxThreads, 1)
         if (!r_ok) return;
         // pixel index inside the segment's (b, g) plane
         const int lp = (int)(it - (long long)(sg.b * a.G + sg.g) * hw);
-        r_ho = lp / a.Wo;
-        r_wo = lp - r_ho * a.Wo;
+        unsigned wo_u;
+        r_ho = (int)fdiv((unsigned)lp, s.fd_wo, wo_u);
+        r_wo = (int)wo_u;
         const long long mi = ((long long)sg.b * hw + lp) * a.G + sg.g;
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
