@@ -180,8 +180,8 @@ dcn_status proj_call(const dcn_params *p, int32_t Cout, const void *x, const voi
         return fail(DCN_ERR_UNSUPPORTED, "the fused contraction takes kh*kw <= 25");
     if (Cout < 8 || Cout > 512 || Cout % 8 != 0)
         return fail(DCN_ERR_UNSUPPORTED, "Cout must be a multiple of 8 in [8, 512] (Cout = %d)", Cout);
-    if ((long long)p->H * p->W >= (1LL << 31) || (long long)p->B * Ho * Wo >= (1LL << 31))
-        return fail(DCN_ERR_UNSUPPORTED, "the fused contraction takes H*W and B*Ho*Wo below 2^31");
+    if ((long long)p->B * p->H * p->W >= (1LL << 31) || (long long)p->B * Ho * Wo >= (1LL << 31))
+        return fail(DCN_ERR_UNSUPPORTED, "the fused contraction takes B*H*W and B*Ho*Wo below 2^31");
     if (p->B == 0) return DCN_OK;
     if (!x || !offset || !mask || !weight || !out)
         return fail(DCN_ERR_NULL, "x, offset, mask, weight and out are required");

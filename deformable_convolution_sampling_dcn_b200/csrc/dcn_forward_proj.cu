@@ -65,6 +65,7 @@ struct ProjParams {
     int cbk;            // K-blocks per kernel point (KB when the points are summed first)
     int per_point;      // 1: deformable convolution, one K-block per (point, channel block)
     int lg_gpb;         // log2 of the groups per K-block (64 / C)
+    int pp_records;     // per-point mode with one record per item (32-item steps)
     FastDiv fd_cbk, fd_howo, fd_wo;  // K-blocks per point, Ho*Wo, Wo
     int n_cta;
     int npad_max;       // largest padded chunk of any CTA (B operand rows)
@@ -298,7 +299,103 @@ __device__ __forceinline__ void gather_step(const ProjParams &p, int ci, long lo
     if (RECORDS) __syncwarp();  // records are rewritten by the next step
 }
 
-template <typename T, int LPI, bool SOFTMAX, int KMAX, bool RECORDS>
+// Per-point records (deformable convolution: every item is one kernel point
+// of one (pixel, group)).  A step is 32 consecutive items of the chunk's flat
+// list.  Lane l first turns item base + l into a record: its four corner
+// pixels (image-wide index, -1 outside the map), its four bilinear weights with
+// the modulation folded in, and where its 16-byte chunks go in the B-operand
+// slot.  Then the LPI lanes of each item gather its channel chunks, IPW items
+// per round, LPI rounds, so every tap is computed once instead of once per lane.
+template <typename T, int LPI, bool SOFTMAX>
+__device__ __forceinline__ void gather_step_pp(const ProjParams &p, int ci, long long c0, FastDiv fd_npx, int total,
+                                               int base, int lane, unsigned char *bring, int slot_bytes,
+                                               float4 *rec_w, int4 *rec_o, int2 *rec_d, const int2 *ktab) {
+    constexpr int V = Storage<T>::kVec;
+    constexpr int IPW = 32 / LPI;
+    const CoreArgs &a = p.a;
+    const int K = a.kh * a.kw;
+    const int GC = a.G * a.C;
+    {
+        // ---- record of item base + lane
+        const int item = base + lane;
+        const bool valid = item < total;
+        const ItemPos ip = item_pos(valid ? item : 0, fd_npx, p);
+        const unsigned pix = (unsigned)(c0 + ip.px);
+        unsigned rem, wo_u;
+        const unsigned b = fdiv(pix, p.fd_howo, rem);
+        const int ho = (int)fdiv(rem, p.fd_wo, wo_u), wo = (int)wo_u;
+        const long long mi = (long long)pix * a.G + ip.g;
+        const T *m_item = static_cast<const T *>(a.mask) + mi * K;
+        const float2 d = load_pair(static_cast<const T *>(a.offset) + (mi * K + ip.k) * 2);
+        float mk = load_scalar(m_item + ip.k);
+        if (SOFTMAX) {
+            float mx = -INFINITY;
+            for (int k = 0; k < K; ++k) mx = fmaxf(mx, load_scalar(m_item + k));
+            float sum = 0.0f;
+            for (int k = 0; k < K; ++k) sum += expf(load_scalar(m_item + k) - mx);
+            mk = expf(mk - mx) * (1.0f / sum);
+        }
+        const int2 kt = ktab[ip.k];
+        const float pxf = fmaf(a.offset_scale, d.x, (float)(wo * a.sw - a.pw + kt.y));
+        const float pyf = fmaf(a.offset_scale, d.y, (float)(ho * a.sh - a.ph + kt.x));
+        const float fy = floorf(pyf), fx = floorf(pxf);
+        const float ly = pyf - fy, lx = pxf - fx;  // NaN for a NaN position
+        const bool nanp = (pxf != pxf) | (pyf != pyf);
+        const bool inmap = (pyf >= -1.0f) & (pyf < (float)a.H) & (pxf >= -1.0f) & (pxf < (float)a.W);
+        const int y0 = inmap ? (int)fy : -2, x0 = inmap ? (int)fx : -2;
+        const bool vy0 = (unsigned)y0 < (unsigned)a.H, vy1 = (unsigned)(y0 + 1) < (unsigned)a.H;
+        const bool vx0 = (unsigned)x0 < (unsigned)a.W, vx1 = (unsigned)(x0 + 1) < (unsigned)a.W;
+        const int r00 = ((int)b * a.H + y0) * a.W + x0;  // B*H*W < 2^31
+        int4 o4 = make_int4(vy0 & vx0 ? r00 : -1, vy0 & vx1 ? r00 + 1 : -1, vy1 & vx0 ? r00 + a.W : -1,
+                            vy1 & vx1 ? r00 + a.W + 1 : -1);
+        const float tx0 = (1.0f - lx) * mk, tx1 = lx * mk;
+        float4 w4 = make_float4(fmaf(-tx0, ly, tx0), fmaf(-tx1, ly, tx1), tx0 * ly, tx1 * ly);
+        if (!(valid & (inmap | nanp))) w4 = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (!valid) o4 = make_int4(-1, -1, -1, -1);
+        rec_w[lane] = w4;  // a NaN position keeps NaN weights and zero-row corners
+        rec_o[lane] = o4;
+        // slot row of the item's K-block and the group's first channel (-1: no item)
+        rec_d[lane] = make_int2(((ci * p.KB + ip.kb) % kBSlots) * slot_bytes + ip.px * 128, valid ? ip.g * a.C : -1);
+    }
+    __syncwarp();
+    // ---- gather: lanes (gi, q) take the 16-byte chunk q of item r * IPW + gi
+    const int gi = lane / LPI, q = lane % LPI;
+    const T *__restrict__ xq = static_cast<const T *>(a.x) + q * V;
+    const unsigned char *zrow = g_zero_row + q * 16;
+#pragma unroll
+    for (int r = 0; r < LPI; ++r) {
+        const int idx = r * IPW + gi;
+        const float4 w = rec_w[idx];
+        const int4 o = rec_o[idx];
+        const int2 dd = rec_d[idx];
+        const T *xb = xq + (dd.y < 0 ? 0 : dd.y);
+        const uint4 v0 = ld_nc16(o.x >= 0 ? (const void *)(xb + (long long)o.x * GC) : (const void *)zrow);
+        const uint4 v1 = ld_nc16(o.y >= 0 ? (const void *)(xb + (long long)o.y * GC) : (const void *)zrow);
+        const uint4 v2 = ld_nc16(o.z >= 0 ? (const void *)(xb + (long long)o.z * GC) : (const void *)zrow);
+        const uint4 v3 = ld_nc16(o.w >= 0 ? (const void *)(xb + (long long)o.w * GC) : (const void *)zrow);
+        float acc[V], f[V];
+        unpack16<T>(v0, f);
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = w.x * f[v];
+        unpack16<T>(v1, f);
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = fmaf(w.y, f[v], acc[v]);
+        unpack16<T>(v2, f);
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = fmaf(w.z, f[v], acc[v]);
+        unpack16<T>(v3, f);
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[v] = fmaf(w.w, f[v], acc[v]);
+        if (dd.y >= 0) {
+            // 16-byte chunk of the item's slot row, swizzled (slot bytes are a multiple of 1024)
+            const int chunk = (dd.y & 63) / V + q;
+            *reinterpret_cast<uint4 *>(bring + dd.x + ((chunk ^ ((dd.x >> 7) & 7)) << 4)) = pack16<T>(acc);
+        }
+    }
+    __syncwarp();  // records are rewritten by the next step
+}
+
+template <typename T, int LPI, bool SOFTMAX, int KMAX, bool RECORDS, bool PP>
 __global__ void __launch_bounds__(kProjThreads, 1)
     core_forward_proj(const __grid_constant__ CUtensorMap wmap, const ProjParams p) {
     constexpr int IPW = 32 / LPI;
@@ -315,10 +412,13 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     unsigned char *bring = smem;
     unsigned char *wst = bring + (size_t)kBSlots * slot_bytes;
     unsigned char *rp = wst + kWStages * kWTileBytes;
-    float4 *rec_w = reinterpret_cast<float4 *>(rp) + (warp < kGatherWarps ? warp : 0) * KMAX * IPW;
-    int4 *rec_o = reinterpret_cast<int4 *>(rp + (RECORDS ? kGatherWarps * KMAX * IPW * 16 : 0)) +
-                  (warp < kGatherWarps ? warp : 0) * KMAX * IPW;
-    rp += RECORDS ? kGatherWarps * KMAX * IPW * 32 : 0;
+    // records per gather warp: one per (item, point) of a step, or one per item of a per-point step
+    constexpr int RECS = PP ? 32 : (RECORDS ? KMAX * IPW : 0);
+    const int wsel = warp < kGatherWarps ? warp : 0;
+    float4 *rec_w = reinterpret_cast<float4 *>(rp) + wsel * RECS;
+    int4 *rec_o = reinterpret_cast<int4 *>(rp + kGatherWarps * RECS * 16) + wsel * RECS;
+    int2 *rec_d = reinterpret_cast<int2 *>(rp + kGatherWarps * RECS * 32) + wsel * RECS;
+    rp += kGatherWarps * RECS * (PP ? 40 : 32);
     int2 *ktab = reinterpret_cast<int2 *>(rp);
     uint64_t *bars = reinterpret_cast<uint64_t *>(ktab + KMAX);
     constexpr int kBars = 2 * kWStages + 2 * kBSlots + 3;
@@ -449,7 +549,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             const int total = per_kb * p.KB;
             const FastDiv fd_npx = make_fastdiv((unsigned)n_px), fd_pkb = make_fastdiv((unsigned)per_kb);
             unsigned fr;
-            const int n_steps = (total + IPW - 1) / IPW;
+            constexpr int SI = PP ? 32 : IPW;  // items per step
+            const int n_steps = (total + SI - 1) / SI;
             int waited = -1;    // slots of K-blocks <= waited are known to be free
             int signaled = 0;   // K-blocks < signaled are handed to the tensor core by this warp
             // wait until the products that read K-block kb's slot before are done
@@ -479,8 +580,8 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             float dx[NT], dy[NT], m[NT];
             if (RECORDS) load_raw<T, LPI, SOFTMAX, NT>(p, c0, fd_npx, total, warp * IPW + ri, k0, dx, dy, m);
             for (int st = warp; st < n_steps; st += kGatherWarps) {
-                const int first = st * IPW;
-                const int last = (first + IPW < total ? first + IPW : total) - 1;
+                const int first = st * SI;
+                const int last = (first + SI < total ? first + SI : total) - 1;
                 // K-blocks before this step's first one hold nothing more of this
                 // warp: hand them over before waiting for any slot, so that every
                 // wait below depends only on K-blocks this warp has already
@@ -500,10 +601,14 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                 const int nxt = st + kGatherWarps;
                 if (RECORDS && nxt < n_steps)
                     load_raw<T, LPI, SOFTMAX, NT>(p, c0, fd_npx, total, nxt * IPW + ri, k0, dx, dy, m);
-                gather_step<T, LPI, SOFTMAX, KMAX, RECORDS, NT>(p, ci, c0, fd_npx, total, first, lane, bring,
-                                                                 slot_bytes, rec_w, rec_o, ktab, cdx, cdy, cm);
+                if constexpr (PP)
+                    gather_step_pp<T, LPI, SOFTMAX>(p, ci, c0, fd_npx, total, first, lane, bring, slot_bytes, rec_w,
+                                                    rec_o, rec_d, ktab);
+                else
+                    gather_step<T, LPI, SOFTMAX, KMAX, RECORDS, NT>(p, ci, c0, fd_npx, total, first, lane, bring,
+                                                                     slot_bytes, rec_w, rec_o, ktab, cdx, cdy, cm);
                 // every K-block before the one this warp's next step starts in is done
-                if (!signal(nxt < n_steps ? (int)fdiv((unsigned)(nxt * IPW), fd_pkb, fr) : p.KB)) {
+                if (!signal(nxt < n_steps ? (int)fdiv((unsigned)(nxt * SI), fd_pkb, fr) : p.KB)) {
                     stop = true;
                     break;
                 }
@@ -547,9 +652,9 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     }
 }
 
-template <typename T, int LPI, bool SOFTMAX, int KMAX, bool RECORDS>
+template <typename T, int LPI, bool SOFTMAX, int KMAX, bool RECORDS, bool PP = false>
 cudaError_t launch_one(const CUtensorMap &map, const ProjParams &p, size_t smem, cudaStream_t stream) {
-    auto kern = core_forward_proj<T, LPI, SOFTMAX, KMAX, RECORDS>;
+    auto kern = core_forward_proj<T, LPI, SOFTMAX, KMAX, RECORDS, PP>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<p.n_cta, kProjThreads, smem, stream>>>(map, p);
@@ -557,15 +662,22 @@ cudaError_t launch_one(const CUtensorMap &map, const ProjParams &p, size_t smem,
 }
 
 // Shared memory of one instance: B ring + weight ring + records + table + barriers, plus alignment slack.
-constexpr size_t proj_smem(int npad_max, int lpi, int kmax, bool records) {
+constexpr size_t proj_smem(int npad_max, int lpi, int kmax, bool records, bool pp = false) {
     return (size_t)kBSlots * npad_max * 128 + (size_t)kWStages * kWTileBytes +
-           (records ? (size_t)kGatherWarps * kmax * (32 / lpi) * 32 : 0) + (size_t)kmax * 8 + 256 + 1024;
+           (pp ? (size_t)kGatherWarps * 32 * 40 : records ? (size_t)kGatherWarps * kmax * (32 / lpi) * 32 : 0) +
+           (size_t)kmax * 8 + 256 + 1024;
 }
 
 template <typename T, int LPI>
 cudaError_t launch_lpi(const CUtensorMap &map, const ProjParams &p, size_t min_smem, cudaStream_t stream) {
     const int K = p.a.kh * p.a.kw;
     auto pick = [&](size_t need) { return need > min_smem ? need : min_smem; };
+    if (p.per_point && p.pp_records) {
+        // one tap per item, built once per item into a record
+        const size_t smem = pick(proj_smem(p.npad_max, LPI, 25, false, true));
+        return p.a.softmax ? launch_one<T, LPI, true, 25, false, true>(map, p, smem, stream)
+                           : launch_one<T, LPI, false, 25, false, true>(map, p, smem, stream);
+    }
     if (p.per_point) {
         // one tap per item: every lane computes its own
         const size_t smem = pick(proj_smem(p.npad_max, LPI, 25, false));
@@ -617,6 +729,13 @@ cudaError_t launch_t(const ProjArgs &pa, cudaStream_t stream) {
     while (cols < p.MB * p.npad_max) cols <<= 1;
     p.tmem_cols = cols;
     p.w_box_rows = pa.Cout < 128 ? pa.Cout : 128;
+    // A per-point step of 32 items must span at most four K-blocks (the slot
+    // ring): every chunk needs at least 11 items per K-block.  A chunk holds
+    // min(range, 128) pixels when its range is at most 128, else at least 64;
+    // every range holds at least floor(P / n_cta) pixels.
+    const long long min_range = p.P / p.n_cta;
+    const long long min_px = min_range > kMaxChunk ? 64 : min_range;
+    p.pp_records = pa.per_point && (min_px << p.lg_gpb) >= 11 ? 1 : 0;
 
     // at least half an SM's shared memory, so that one CTA owns the SM's
     // tensor memory (the largest instance needs about 200 KB)

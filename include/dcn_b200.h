@@ -123,7 +123,7 @@ dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offs
  * result once.  The core never reaches device memory.
  * Supported: fp16 and bf16 (fp32 returns DCN_ERR_UNSUPPORTED), C <= 64 with
  * G*C a multiple of 64 up to 512, kh*kw <= 25, Cout a multiple of 8 in
- * [8, 512], H*W and B*Ho*Wo below 2^31; both mask modes.  x, weight and out
+ * [8, 512], B*H*W and B*Ho*Wo below 2^31; both mask modes.  x, weight and out
  * 16-byte aligned, offset 4-byte, mask and bias 2-byte.  A NaN sampling
  * position makes every output channel of its pixel NaN.
  */

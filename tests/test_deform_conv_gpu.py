@@ -46,6 +46,9 @@ SMALL = [
     (1, 12, 13, 8, 8, 96, "bf16", dict(kh=5, kw=5, pad=2)),            # 25 points, C = 8
     (1, 15, 19, 16, 32, 64, "f16", dict(stride=2, pad=2, dil=2, oob=0.1)),
     (1, 4, 5, 16, 32, 64, "f16", {}),                                  # 20 pixels: small chunks, 72 K-blocks
+    # fewer than 11 items per K-block in a chunk: every lane computes its own tap
+    (1, 3, 3, 8, 64, 64, "f16", {}),
+    (1, 2, 5, 4, 64, 24, "bf16", dict(softmax=True)),
 ]
 
 

@@ -109,6 +109,23 @@ def test_projection(i, cuda_dev):
     assert_close_fwd(out, oracle.pointwise_projection(core, inp["weight"], inp["bias"]), f"random proj {i}")
 
 
+@pytest.mark.parametrize("i", range(12))
+def test_deform_conv(i, cuda_dev):
+    import deformable_convolution_sampling_dcn_b200 as d
+
+    shape, cout = draw_proj(100 + i)
+    inp = si.core_inputs(shape, 9000 + i)
+    inp.update(si.deform_conv_weights(shape.K, shape.G * shape.C, cout, shape.dtype, 9500 + i))
+    t = {k: v.to(cuda_dev) for k, v in inp.items()}
+    out = d.dcn_deform_conv_forward(t["x"], t["offset"], t["mask"], t["weight"], t["bias"], group=shape.G,
+                                    **geo(shape))
+    torch.cuda.synchronize()
+    assert d._binding.take_device_error() == 0
+    ref = oracle.deform_conv_forward(inp["x"], inp["offset"], inp["mask"], inp["weight"], inp["bias"], G=shape.G,
+                                     **ogeo(shape))
+    assert_close_fwd(out, ref, f"random deform conv {i}")
+
+
 def draw_roi(i):
     r = np.random.default_rng(8000 + i)
     dt = ["f32", "f16", "bf16"][r.integers(3)]
