@@ -231,12 +231,22 @@ def run_ours(args, world, rank, local):
     achieved = bytes_per_launch / step_s / 1e9
     peak, peak_kind = peaks()
     traffic = None
+    issue = None
     if os.path.exists(TRAFFIC_FILE):
         with open(TRAFFIC_FILE) as f:
             tr = json.load(f)
         ent = tr.get("dcnv4_p4_forward")
         if ent and ent.get("kernel_hash") == kernel_hash():
             traffic = ent["dram_bytes_per_launch"]
+            insts = ent.get("warp_instructions_per_launch")
+            if insts and clocks.get("sm_mhz"):
+                # the ceiling that binds this gather: one warp instruction per
+                # scheduler per clock (148 SMs x 4 schedulers at the sampled clock)
+                ceil_t = torch.cuda.get_device_properties(dev).multi_processor_count * 4 * clocks["sm_mhz"] * 1e6
+                ach_t = insts / step_s
+                issue = {"warp_instructions_per_launch": insts, "achieved": round(ach_t / 1e12, 4),
+                         "ceiling": round(ceil_t / 1e12, 4), "unit": "T warp-instructions/s",
+                         "frac": round(ach_t / ceil_t, 4)}
 
     # end to end through the public API with host buffers (pinned), copies timed
     e2e = measure_e2e(dcn, shape, inp, dev, stream, min(K, args.e2e_steps), barrier, world)
@@ -267,7 +277,7 @@ def run_ours(args, world, rank, local):
                          "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
                          else "fallback 6.65 TB/s",
                          "algorithmic_bytes_per_launch": bytes_per_launch,
-                         "kernel": "dcn_core_forward (one launch per step)"},
+                         "kernel": "dcn_core_forward (one launch per step)", "issue": issue},
             "clocks": clocks,
             "e2e": e2e,
             "gpu_launches": K,
