@@ -464,17 +464,21 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         // ---- weight tiles, in the order the MMA thread consumes them
         if (lane == 0) {
             int it = 0;
+            uint32_t s = 0, pass = 0;  // stage of the next tile and how often the ring has wrapped
             const uint32_t tx = (uint32_t)p.w_box_rows * 128u;
             for (int ci = 0; ci < n_chunks && !*abort_flag; ++ci)
                 for (int kb = 0; kb < p.KB && !*abort_flag; ++kb)
                     for (int mb = 0; mb < p.MB; ++mb, ++it) {
-                        const int s = it % kWStages, u = it / kWStages;
-                        if (u >= 1 && !wait_or_abort(wempty + 8 * s, (u - 1) & 1, abort_flag)) {
+                        if (pass >= 1 && !wait_or_abort(wempty + 8 * s, (pass - 1) & 1, abort_flag)) {
                             raise_abort(abort_flag, p.err);
                             break;
                         }
                         mbar_arrive_expect_tx(wfull + 8 * s, tx);
                         tma_load_2d(wst_a + s * kWTileBytes, &wmap, wfull + 8 * s, kb * 64, mb * 128);
+                        if (++s == kWStages) {
+                            s = 0;
+                            ++pass;
+                        }
                     }
             // drain: the last load issued into each stage has landed
             for (int j = it - 1; j >= 0 && j >= it - kWStages; --j)
@@ -484,7 +488,14 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     } else if (warp == kMmaWarp) {
         // ---- tensor-core products, one thread
         if (lane == 0) {
-            int it = 0;
+            // One thread issues every product, so its own instruction latency paces
+            // the tensor core: between products it only steps counters and adds
+            // precomputed descriptor offsets (no division, no descriptor rebuild).
+            uint32_t ws = 0, wph = 0;  // weight stage of the next tile, its phase parity
+            uint32_t bsl = 0, bph = 0; // B slot of the next K-block, its phase parity
+            // descriptors are linear in the address (start address >> 4 in the low field)
+            const uint64_t adesc0 = smem_desc_sw128(wst_a), bdesc0 = smem_desc_sw128(bring_a);
+            const uint32_t slot_step = (uint32_t)slot_bytes >> 4, stage_step = kWTileBytes >> 4;
             bool issued = false;
             const int fmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
             for (int ci = 0; ci < n_chunks && !*abort_flag; ++ci) {
@@ -498,31 +509,44 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                for (int kb = 0; kb < p.KB && !*abort_flag; ++kb) {
-                    const int t = ci * p.KB + kb, bs = t % kBSlots;
-                    if (!wait_or_abort(kready + 8 * bs, (t / kBSlots) & 1, abort_flag)) {
-                        raise_abort(abort_flag, p.err);
+                bool ok = true;
+                for (int kb = 0; kb < p.KB && ok; ++kb) {
+                    if (!wait_or_abort(kready + 8 * bsl, bph, abort_flag)) {
+                        ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t b_kb = bring_a + (uint32_t)(bs * slot_bytes);
-                    for (int mb = 0; mb < p.MB; ++mb, ++it) {
-                        const int s = it % kWStages;
-                        if (!wait_or_abort(wfull + 8 * s, (it / kWStages) & 1, abort_flag)) {
-                            raise_abort(abort_flag, p.err);
+                    const uint64_t bdesc = bdesc0 + bsl * slot_step;
+                    uint32_t dcol = tmem;
+                    for (int mb = 0; mb < p.MB; ++mb, dcol += (uint32_t)npad) {
+                        if (!wait_or_abort(wfull + 8 * ws, wph, abort_flag)) {
+                            ok = false;
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t a_s = wst_a + s * kWTileBytes;
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            mma_f16(tmem + (uint32_t)(mb * npad), smem_desc_sw128(a_s + k * 32),
-                                    smem_desc_sw128(b_kb + k * 32), idesc, (kb | k) != 0);
+                        // k-steps of 16 elements = 32 bytes = 2 descriptor units
+                        const uint64_t adesc = adesc0 + ws * stage_step;
+                        mma_f16(dcol, adesc, bdesc, idesc, kb != 0);
+                        mma_f16(dcol, adesc + 2, bdesc + 2, idesc, 1u);
+                        mma_f16(dcol, adesc + 4, bdesc + 4, idesc, 1u);
+                        mma_f16(dcol, adesc + 6, bdesc + 6, idesc, 1u);
                         issued = true;
-                        mma_commit(wempty + 8 * s);  // weight stage free once these products are done
+                        mma_commit(wempty + 8 * ws);  // weight stage free once these products are done
+                        if (++ws == kWStages) {
+                            ws = 0;
+                            wph ^= 1u;
+                        }
                     }
-                    if (*abort_flag) break;
-                    mma_commit(bfree + 8 * bs);  // B slot free once this K-block's products are done
+                    if (!ok) break;
+                    mma_commit(bfree + 8 * bsl);  // B slot free once this K-block's products are done
+                    if (++bsl == kBSlots) {
+                        bsl = 0;
+                        bph ^= 1u;
+                    }
+                }
+                if (!ok) {
+                    raise_abort(abort_flag, p.err);
+                    break;
                 }
                 if (*abort_flag) break;
                 mma_commit(dfull);  // accumulators of this chunk complete
