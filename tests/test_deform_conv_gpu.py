@@ -73,6 +73,18 @@ def test_without_bias_and_regular_conv_limit(cuda_dev):
     assert_close_fwd(out, conv.permute(0, 2, 3, 1).numpy(), "deform conv vs conv2d")
 
 
+@pytest.mark.parametrize("B,H,W,G,C,cout,dt,softmax", [
+    (4, 70, 70, 2, 32, 64, "f16", False),     # 19,600 pixels: two chunks per CTA
+    (4, 100, 100, 4, 16, 32, "bf16", True),   # 40,000 pixels: three chunks per CTA
+])
+def test_several_chunks_per_cta(B, H, W, G, C, cout, dt, softmax, cuda_dev):
+    """More than 128 pixels per CTA: the per-point work list, the weight stream and
+    the accumulators are reused chunk after chunk."""
+    shape, inp = case(B, H, W, G, C, cout, dt, seed=90 + B + H, softmax=softmax)
+    out, ref = run(shape, inp, cuda_dev)
+    assert_close_fwd(out, ref, f"deform conv {B}x{H}x{W}")
+
+
 def test_dcnv2_p4_full_size(cuda_dev):
     """DCNv2-style deformable convolution at the P4 shape: B=8, 40x40, 512 input
     channels as 16 deformable groups of 32, 3x3, 256 output channels, fp16."""
