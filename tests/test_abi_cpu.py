@@ -179,3 +179,6 @@ def test_deform_conv_checks(lib):
     assert f(ctypes.byref(p), 100, 16, 16, 16, 16, None, 16, None) == B.DCN_ERR_UNSUPPORTED
     assert f(ctypes.byref(params(G=16, C=32, dtype=0)), 64, 16, 16, 16, 16, None, 16, None) == B.DCN_ERR_UNSUPPORTED
     assert f(ctypes.byref(params(B=0, G=16, C=32)), 64, None, None, None, None, None, None, None) == B.DCN_OK
+    # B*H*W = 2^31 input pixels (corner indices are 32-bit) while B*Ho*Wo = 2^29
+    big = params(B=2048, H=1024, W=1024, G=16, C=32, stride_h=2, stride_w=2)
+    assert f(ctypes.byref(big), 64, 16, 16, 16, 16, None, 16, None) == B.DCN_ERR_UNSUPPORTED
