@@ -51,6 +51,7 @@ constexpr int kMmaWarp = kGatherWarps + 1;
 constexpr int kProjThreads = (kGatherWarps + 2) * 32;
 constexpr int kWStages = 4;
 constexpr int kWTileBytes = 128 * 128;  // 128 rows x 64 elements x 2 bytes
+constexpr int kWTileBytesSwap = 256 * 128;  // 256 output channels x 64 elements x 2 bytes
 constexpr int kMaxChunk = 128;          // pixels per chunk (MMA N <= 128)
 constexpr int kBSlots = 4;             // B-operand ring: K-blocks in flight
 constexpr uint64_t kProjWaitNs = 1000000000ull;
@@ -70,7 +71,8 @@ struct ProjParams {
     int n_cta;
     int npad_max;       // largest padded chunk of any CTA (B operand rows)
     int tmem_cols;      // allocated tensor-memory columns (power of two >= 32)
-    int w_box_rows;     // rows per weight TMA box (min(Cout, 128))
+    int w_box_rows;     // rows per weight TMA box: min(Cout, 128), or min(Cout16, 256) when swapped
+    int cout16;         // Cout rounded up to a multiple of 16
     unsigned int *err;
 };
 
@@ -404,14 +406,20 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 
     extern __shared__ unsigned char smem_raw[];
     // 1024-byte aligned base (the swizzle pattern repeats every 1024 bytes):
-    // [B-operand ring: kBSlots x npad_max x 128][weight ring: kWStages x 16 KB]
+    // [sample ring: kBSlots x npad_max x 128][weight ring: kWStages x 16 KB (32 KB swapped)]
     // [records: weights, corners][kernel-point table][barriers, tensor-memory address, abort flag]
     const uint32_t raw_a = smem_u32(smem_raw);
     unsigned char *smem = smem_raw + (((raw_a + 1023u) & ~1023u) - raw_a);
     const int slot_bytes = p.npad_max * 128;
     unsigned char *bring = smem;
     unsigned char *wst = bring + (size_t)kBSlots * slot_bytes;
-    unsigned char *rp = wst + kWStages * kWTileBytes;
+    // Per-point records swap the roles: the sampled pixels are the M = 128 operand
+    // and up to 256 output channels of the weight the N operand, so that each
+    // weight tile feeds products of N = 256 (a 4-product tile costs a fixed few
+    // hundred cycles of hand-over, which only products of N >= 128 cover).
+    constexpr bool SWAP = PP;
+    constexpr int WTILE = SWAP ? kWTileBytesSwap : kWTileBytes;
+    unsigned char *rp = wst + kWStages * WTILE;
     // records per gather warp: one per (item, point) of a step, or one per item of a per-point step
     constexpr int RECS = PP ? 32 : (RECORDS ? KMAX * IPW : 0);
     const int wsel = warp < kGatherWarps ? warp : 0;
@@ -474,7 +482,7 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                             break;
                         }
                         mbar_arrive_expect_tx(wfull + 8 * s, tx);
-                        tma_load_2d(wst_a + s * kWTileBytes, &wmap, wfull + 8 * s, kb * 64, mb * 128);
+                        tma_load_2d(wst_a + s * WTILE, &wmap, wfull + 8 * s, kb * 64, mb * (SWAP ? 256 : 128));
                         if (++s == kWStages) {
                             s = 0;
                             ++pass;
@@ -495,14 +503,18 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             uint32_t bsl = 0, bph = 0; // B slot of the next K-block, its phase parity
             // descriptors are linear in the address (start address >> 4 in the low field)
             const uint64_t adesc0 = smem_desc_sw128(wst_a), bdesc0 = smem_desc_sw128(bring_a);
-            const uint32_t slot_step = (uint32_t)slot_bytes >> 4, stage_step = kWTileBytes >> 4;
+            const uint32_t slot_step = (uint32_t)slot_bytes >> 4, stage_step = WTILE >> 4;
             bool issued = false;
             const int fmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
             for (int ci = 0; ci < n_chunks && !*abort_flag; ++ci) {
                 long long c0, c1;
                 chunk_range(r0, r1, ci, n_chunks, c0, c1);
                 const int npad = ((int)(c1 - c0) + 15) & ~15;
-                const uint32_t idesc = instr_desc_f16(fmt, npad);
+                // swapped: N = 256 output channels per tile, the last tile the rest
+                const int n_last = p.cout16 - 256 * (p.MB - 1);
+                const uint32_t idesc = instr_desc_f16(fmt, SWAP ? (p.MB > 1 ? 256 : n_last) : npad);
+                const uint32_t idesc_last = SWAP ? instr_desc_f16(fmt, n_last) : idesc;
+                const uint32_t dstep = SWAP ? 256u : (uint32_t)npad;
                 // the epilogue has read the previous chunk's accumulators
                 if (ci > 0 && !wait_or_abort(tempty, (ci - 1) & 1, abort_flag)) {
                     raise_abort(abort_flag, p.err);
@@ -518,18 +530,26 @@ __global__ void __launch_bounds__(kProjThreads, 1)
                     tc_fence_after();
                     const uint64_t bdesc = bdesc0 + bsl * slot_step;
                     uint32_t dcol = tmem;
-                    for (int mb = 0; mb < p.MB; ++mb, dcol += (uint32_t)npad) {
+                    for (int mb = 0; mb < p.MB; ++mb, dcol += dstep) {
                         if (!wait_or_abort(wfull + 8 * ws, wph, abort_flag)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         // k-steps of 16 elements = 32 bytes = 2 descriptor units
-                        const uint64_t adesc = adesc0 + ws * stage_step;
-                        mma_f16(dcol, adesc, bdesc, idesc, kb != 0);
-                        mma_f16(dcol, adesc + 2, bdesc + 2, idesc, 1u);
-                        mma_f16(dcol, adesc + 4, bdesc + 4, idesc, 1u);
-                        mma_f16(dcol, adesc + 6, bdesc + 6, idesc, 1u);
+                        const uint64_t wdesc = adesc0 + ws * stage_step;
+                        if (SWAP) {  // D[pixel, channel] += samples . weight^T
+                            const uint32_t id = mb + 1 < p.MB ? idesc : idesc_last;
+                            mma_f16(dcol, bdesc, wdesc, id, kb != 0);
+                            mma_f16(dcol, bdesc + 2, wdesc + 2, id, 1u);
+                            mma_f16(dcol, bdesc + 4, wdesc + 4, id, 1u);
+                            mma_f16(dcol, bdesc + 6, wdesc + 6, id, 1u);
+                        } else {     // D[channel, pixel] += weight . samples^T
+                            mma_f16(dcol, wdesc, bdesc, idesc, kb != 0);
+                            mma_f16(dcol, wdesc + 2, bdesc + 2, idesc, 1u);
+                            mma_f16(dcol, wdesc + 4, bdesc + 4, idesc, 1u);
+                            mma_f16(dcol, wdesc + 6, bdesc + 6, idesc, 1u);
+                        }
                         issued = true;
                         mma_commit(wempty + 8 * ws);  // weight stage free once these products are done
                         if (++ws == kWStages) {
@@ -646,6 +666,32 @@ __global__ void __launch_bounds__(kProjThreads, 1)
             }
             tc_fence_after();
             const int quad = warp & 3, part = warp >> 2;
+            if (SWAP) {
+                // tensor-memory lane = pixel of the chunk, column = output channel
+                const int px = 32 * quad + lane;
+                if (32 * quad < n_px) {
+                    T *orow = out + (c0 + (px < n_px ? px : 0)) * p.Cout;
+                    for (int cc = part; cc < p.cout16 / 16; cc += kGatherWarps / 4) {
+                        float v[16];
+                        tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(cc * 16), v);
+                        const int o0 = cc * 16;
+                        if (px < n_px) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                if (o0 + j < p.Cout) v[j] += bias ? load_scalar(bias + o0 + j) : 0.0f;
+                            if (o0 + 16 <= p.Cout) {  // rows are 16-byte aligned (Cout % 8 == 0)
+                                uint4 *dst = reinterpret_cast<uint4 *>(orow + o0);
+                                dst[0] = pack16<T>(v);
+                                dst[1] = pack16<T>(v + 8);
+                            } else {
+#pragma unroll
+                                for (int j = 0; j < 16; ++j)
+                                    if (o0 + j < p.Cout) orow[o0 + j] = from_f32<T>(v[j]);
+                            }
+                        }
+                    }
+                }
+            } else
             for (int blk = part; blk < npad / 16; blk += kGatherWarps / 4) {
                 for (int mb = 0; mb < p.MB; ++mb) {
                     float v[16];
@@ -687,7 +733,7 @@ cudaError_t launch_one(const CUtensorMap &map, const ProjParams &p, size_t smem,
 
 // Shared memory of one instance: B ring + weight ring + records + table + barriers, plus alignment slack.
 constexpr size_t proj_smem(int npad_max, int lpi, int kmax, bool records, bool pp = false) {
-    return (size_t)kBSlots * npad_max * 128 + (size_t)kWStages * kWTileBytes +
+    return (size_t)kBSlots * npad_max * 128 + (size_t)kWStages * (pp ? kWTileBytesSwap : kWTileBytes) +
            (pp ? (size_t)kGatherWarps * 32 * 40 : records ? (size_t)kGatherWarps * kmax * (32 / lpi) * 32 : 0) +
            (size_t)kmax * 8 + 256 + 1024;
 }
@@ -748,11 +794,6 @@ cudaError_t launch_t(const ProjArgs &pa, cudaStream_t stream) {
     // every chunk holds at most min(range, 128) pixels, and no range exceeds
     // ceil(P / n_cta)
     const long long max_range = (p.P + p.n_cta - 1) / p.n_cta;
-    p.npad_max = (int)(((max_range < kMaxChunk ? max_range : kMaxChunk) + 15) & ~15LL);
-    int cols = 32;
-    while (cols < p.MB * p.npad_max) cols <<= 1;
-    p.tmem_cols = cols;
-    p.w_box_rows = pa.Cout < 128 ? pa.Cout : 128;
     // A per-point step of 32 items must span at most four K-blocks (the slot
     // ring): every chunk needs at least 11 items per K-block.  A chunk holds
     // min(range, 128) pixels when its range is at most 128, else at least 64;
@@ -760,6 +801,20 @@ cudaError_t launch_t(const ProjArgs &pa, cudaStream_t stream) {
     const long long min_range = p.P / p.n_cta;
     const long long min_px = min_range > kMaxChunk ? 64 : min_range;
     p.pp_records = pa.per_point && (min_px << p.lg_gpb) >= 11 ? 1 : 0;
+    p.cout16 = (pa.Cout + 15) & ~15;
+    int cols = 32;
+    if (p.pp_records) {
+        // swapped products: 128 sample rows (M), output channels in tiles of 256 (N)
+        p.npad_max = kMaxChunk;
+        p.MB = (p.cout16 + 255) / 256;
+        p.w_box_rows = p.cout16 < 256 ? p.cout16 : 256;
+        while (cols < p.cout16) cols <<= 1;
+    } else {
+        p.npad_max = (int)(((max_range < kMaxChunk ? max_range : kMaxChunk) + 15) & ~15LL);
+        p.w_box_rows = pa.Cout < 128 ? pa.Cout : 128;
+        while (cols < p.MB * p.npad_max) cols <<= 1;
+    }
+    p.tmem_cols = cols;
 
     // at least half an SM's shared memory, so that one CTA owns the SM's
     // tensor memory (the largest instance needs about 200 KB)
