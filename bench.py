@@ -555,10 +555,22 @@ def cpu_baseline(seconds: float):
         el = time.perf_counter() - t0
         if el >= seconds:
             break
+    # the same oracle on one core, for a shorter while
+    oracle.set_threads(1)
+    reps1, t1 = 0, time.perf_counter()
+    while True:
+        oracle.dcn_forward(x, off, m, G=shape.G)
+        reps1 += 1
+        el1 = time.perf_counter() - t1
+        if el1 >= seconds / 5:
+            break
+    oracle.set_threads(n)
     return {"value": round(shape.samples * reps / el / 1e9, 5), "unit": "Gsamples/s", "cores": n,
             "kind": "oracle",
             "sample": f"{reps} whole DCNv4-P4 batches (B=8, {shape.samples} samples each) in {el:.1f} s, "
-                      f"fp64 C loops, OpenMP over (b, output row)"}
+                      f"fp64 C loops, OpenMP over (b, output row)",
+            "single_core": {"value": round(shape.samples * reps1 / el1 / 1e9, 5), "unit": "Gsamples/s",
+                            "sample": f"{reps1} whole batches in {el1:.1f} s on 1 thread"}}
 
 
 def run_reference(args, world, rank):
