@@ -679,5 +679,20 @@ def pin_dconv_regular_conv(lib):
         assert np.allclose(out, ref.permute(0, 2, 3, 1).numpy(), rtol=0, atol=1e-11), "deform conv vs conv2d"
 
 
-DCONV_PINS = [pin_dconv_torchvision, pin_dconv_regular_conv]
+def pin_dconv_softmax_vs_raw(lib):
+    """Softmax mode equals raw mode fed with scipy's softmax of the logits over the
+    K points of each (pixel, group)."""
+    from scipy.special import softmax
+
+    x, w, b = _dconv_case(430, B=1, H=6, W=7, G=2, C=3, cout=3)
+    Ho, Wo = oracle.out_hw(6, 7, 3, 3, 1, 1, 1, 1, 1, 1)
+    rng = np.random.default_rng(431)
+    off = rng.standard_normal((1, Ho, Wo, 2, 9, 2)) * 1.5
+    logits = rng.standard_normal((1, Ho, Wo, 2, 9)) * 2.0
+    a = oracle.deform_conv_forward(x, off, logits, w, b, G=2, softmax=True, lib=lib)
+    r = oracle.deform_conv_forward(x, off, softmax(logits, axis=-1), w, b, G=2, softmax=False, lib=lib)
+    assert np.allclose(a, r, rtol=0, atol=1e-12), "deform conv softmax vs raw"
+
+
+DCONV_PINS = [pin_dconv_torchvision, pin_dconv_regular_conv, pin_dconv_softmax_vs_raw]
 ALL_PINS = ALL_PINS + DCONV_PINS

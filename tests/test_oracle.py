@@ -120,6 +120,8 @@ MUTATIONS = [
     ("for (int c = 0; c < C; ++c) ck[c] += m[k] * Gq * xq[c];", "for (int c = 0; c < C; ++c) ck[c] += Gq * xq[c];",
      0, pins.DCONV_PINS),
     ("double acc = bias ? bias[o] : 0.0;", "double acc = 0.0;", 0, pins.DCONV_PINS),
+    # the softmax flag ignored (raw modulation always)
+    ("modulation(mask + item * K, K, softmax, m);", "modulation(mask + item * K, K, 0, m);", 0, pins.DCONV_PINS),
     ("double s = bias ? bias[o] : 0.0;", "double s = 0.0;", 0, pins.PROJ_PINS),
     ("double s = bias ? bias[o] : 0.0;", "double s = bias ? bias[0] : 0.0;", 0, pins.PROJ_PINS),
 ]
