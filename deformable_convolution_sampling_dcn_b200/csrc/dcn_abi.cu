@@ -143,7 +143,7 @@ dcn_status dcn_core_output_hw(const dcn_params *p, int32_t *Ho, int32_t *Wo) {
 
 dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offset, const void *mask,
                             void *out, dcn_stream_t stream) {
-    int Ho, Wo;
+    int Ho = 0, Wo = 0;
     dcn_status s = check_core(p, &Ho, &Wo);
     if (s != DCN_OK) return s;
     if (p->B == 0) return DCN_OK;
@@ -167,7 +167,7 @@ namespace {
 dcn_status proj_call(const dcn_params *p, int32_t Cout, const void *x, const void *offset, const void *mask,
                      const void *weight, const void *bias, void *out, dcn_stream_t stream, bool per_point,
                      const char *what) {
-    int Ho, Wo;
+    int Ho = 0, Wo = 0;
     dcn_status s = check_core(p, &Ho, &Wo);
     if (s != DCN_OK) return s;
     if (p->dtype != DCN_F16 && p->dtype != DCN_BF16)
@@ -216,7 +216,7 @@ dcn_status dcn_deform_conv_forward(const dcn_params *p, int32_t Cout, const void
 dcn_status dcn_core_backward(const dcn_params *p, const void *x, const void *offset, const void *mask,
                              const void *grad_out, void *grad_x, void *grad_offset, void *grad_mask,
                              dcn_stream_t stream) {
-    int Ho, Wo;
+    int Ho = 0, Wo = 0;
     dcn_status s = check_core(p, &Ho, &Wo);
     if (s != DCN_OK) return s;
     if (p->B == 0) return DCN_OK;
