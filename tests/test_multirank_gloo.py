@@ -83,3 +83,22 @@ def test_two_gloo_ranks_shard_the_batch():
     assert fwd_ok and bwd_ok
     assert slowest == 2.0
     assert ranges == [(0, 3), (3, 5)]
+
+
+def test_reference_arm_under_two_ranks(tmp_path):
+    """bench.py --impl reference launched as two ranks: rank 0 alone prints one
+    JSON line, the other rank exits 0 without work."""
+    import json
+    import subprocess
+
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--gpus", "2", "--steps", "3", "--warmup", "3"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
