@@ -54,6 +54,17 @@ def test_golden_aggregation(oracle_lib):
     assert out.item() == ex["expected"]
 
 
+def test_golden_deform_conv(oracle_lib):
+    ex = json.load(open(GOLDEN))["deform_conv"]
+    x = np.array(ex["x"], dtype=np.float64).reshape(1, 1, 3, 1)
+    off = np.array(ex["offset_dx_dy"], dtype=np.float64).reshape(1, 1, 2, 1, 2, 2)
+    mask = np.array(ex["mask"], dtype=np.float64).reshape(1, 1, 2, 1, 2)
+    w = np.array(ex["weight_out_point"], dtype=np.float64).reshape(2, 2, 1)
+    b = np.array(ex["bias"], dtype=np.float64)
+    out = oracle.deform_conv_forward(x, off, mask, w, b, G=1, kh=1, kw=2, pad=(0, 0), lib=oracle_lib)
+    assert np.array_equal(out.reshape(2, 2), np.array(ex["expected_out_pixel_channel"]))
+
+
 def test_nan_position_propagates(oracle_lib):
     """A sampling position that is not a number poisons its (pixel, group)."""
     x = np.ones((1, 4, 4, 2 * 3))
