@@ -65,6 +65,16 @@ def test_golden_deform_conv(oracle_lib):
     assert np.array_equal(out.reshape(2, 2), np.array(ex["expected_out_pixel_channel"]))
 
 
+def test_golden_roi_pool(oracle_lib):
+    ex = json.load(open(GOLDEN))["roi_pool"]
+    x = np.array(ex["x_rows"], dtype=np.float64).reshape(1, 2, 4, 1)
+    rois = np.array([ex["roi"]], dtype=np.float32)
+    off = np.array(ex["offset_dx_dy"], dtype=np.float32).reshape(1, 1, 1, 2)
+    out = oracle.roi_pool_forward(x, rois, off, pooled=(1, 1), sampling=2, spatial_scale=1.0, gamma=0.25,
+                                  lib=oracle_lib)
+    assert out.item() == ex["expected"]
+
+
 def test_nan_position_propagates(oracle_lib):
     """A sampling position that is not a number poisons its (pixel, group)."""
     x = np.ones((1, 4, 4, 2 * 3))
