@@ -75,6 +75,24 @@ def test_golden_roi_pool(oracle_lib):
     assert out.item() == ex["expected"]
 
 
+def test_golden_core_backward(oracle_lib):
+    ex = json.load(open(GOLDEN))["core_backward"]
+    x = np.array(ex["x_rows"], dtype=np.float64).reshape(1, 2, 2, 1)
+    off = np.zeros((1, 2, 2, 1, 1, 2))
+    off[0, 0, 0, 0, 0] = ex["offset_dx_dy_pixel00"]
+    mask = np.zeros((1, 2, 2, 1, 1))
+    mask[0, 0, 0, 0, 0] = ex["mask_pixel00"]
+    go = np.zeros((1, 2, 2, 1))
+    go[0, 0, 0, 0] = ex["grad_out_pixel00"]
+    g = oracle.dcn_backward(x, off, mask, go, G=1, kh=1, kw=1, pad=(0, 0), lib=oracle_lib)
+    e = ex["expected"]
+    assert g["grad_mask"][0, 0, 0, 0, 0] == e["grad_mask_pixel00"]
+    assert g["grad_offset"][0, 0, 0, 0, 0, 0] == e["grad_dx_pixel00"]
+    assert g["grad_offset"][0, 0, 0, 0, 0, 1] == e["grad_dy_pixel00"]
+    assert np.array_equal(g["grad_x"].reshape(2, 2), np.array(e["grad_x_rows"]))
+    assert np.count_nonzero(g["grad_offset"]) == 2 and np.count_nonzero(g["grad_mask"]) == 1
+
+
 def test_nan_position_propagates(oracle_lib):
     """A sampling position that is not a number poisons its (pixel, group)."""
     x = np.ones((1, 4, 4, 2 * 3))
