@@ -1,0 +1,28 @@
+"""The committed profile records match the sources they describe: the DRAM
+traffic and instruction count that bench.py reports for the timed forward kernel
+are used only while the kernel's sources hash to the recorded value, so a kernel
+edit without a new capture shows up here (and as a null `traffic` in the bench
+line)."""
+import json
+import os
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_traffic_record_matches_kernel_sources():
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        ent = json.load(f)["dcnv4_p4_forward"]
+    assert ent["kernel_hash"] == bench.kernel_hash()
+    assert ent["kernel_sources"] == [os.path.basename(p) for p in bench.KERNEL_SOURCES]
+    assert ent["dram_bytes_per_launch"] == ent["dram_bytes_read"] + ent["dram_bytes_write"]
+    assert ent["warp_instructions_per_launch"] > 0
+
+
+def test_profiles_give_their_commands():
+    d = os.path.join(ROOT, "profiles")
+    for name in os.listdir(d):
+        if name.endswith(".md"):
+            text = open(os.path.join(d, name), encoding="utf-8").read()
+            assert "ncu " in text and "--clock-control none" in text, name
