@@ -233,7 +233,8 @@ def roi_pool_forward(x, rois, offset, *, pooled=(7, 7), sampling=2, spatial_scal
                      gamma: float = 0.1, lib=None) -> np.ndarray:
     """out [N, PH, PW, C] (fp64) of deformable RoI pooling over x [B, H, W, C].
 
-    rois [N, 5] (batch, x1, y1, x2, y2) and offset [N, PH, PW, 2] are fp32."""
+    rois [N, 5] (batch, x1, y1, x2, y2) and offset [N, PH, PW, 2] are fp32.  A
+    region whose batch index lies outside [0, B) (or is NaN) pools to zeros."""
     lib = lib or load()
     x = _f64(x)
     B, H, W, C = x.shape
@@ -244,7 +245,6 @@ def roi_pool_forward(x, rois, offset, *, pooled=(7, 7), sampling=2, spatial_scal
     N = r.shape[0]
     PH, PW = pooled
     assert r.shape == (N, 5) and o.shape == (N, PH, PW, 2)
-    assert np.all((r[:, 0] >= 0) & (r[:, 0] < B) & (r[:, 0] == np.floor(r[:, 0])))
     out = np.empty((N, PH, PW, C), dtype=np.float64)
     lib.oracle_roi_pool_forward(B, H, W, C, N, PH, PW, int(sampling), float(spatial_scale), float(gamma),
                                 _ptr(x, ctypes.c_double), _ptr(r, ctypes.c_float), _ptr(o, ctypes.c_float),

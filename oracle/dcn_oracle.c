@@ -494,6 +494,13 @@ void oracle_roi_pool_forward(int B, int H, int W, int C, int N, int PH, int PW, 
 #pragma omp parallel for schedule(static)
     for (int n = 0; n < N; ++n) {
         const float *r = rois + (size_t)n * 5;
+        /* A batch index that names no image of the input (outside [0, B), or
+         * not a number) reads nothing: every bin of the region is zero.
+         * Inside the range the index is the integer part of the value. */
+        if (!(r[0] >= 0.0f && r[0] < (float)B)) {
+            for (size_t e = 0; e < (size_t)PH * PW * C; ++e) out[(size_t)n * PH * PW * C + e] = 0.0;
+            continue;
+        }
         const int b = (int)r[0];
         const float x1 = r[1] * spatial_scale, y1 = r[2] * spatial_scale;
         const float x2 = r[3] * spatial_scale, y2 = r[4] * spatial_scale;
@@ -532,5 +539,4 @@ void oracle_roi_pool_forward(int B, int H, int W, int C, int N, int PH, int PW, 
                 for (int c = 0; c < C; ++c) y[c] = not_a_number ? NAN : y[c] / (double)(S * S);
             }
     }
-    (void)B;
 }

@@ -535,6 +535,26 @@ def pin_roi_brute_force(lib):
         assert np.allclose(out, ref, rtol=0, atol=1e-12), "roi brute force"
 
 
+def pin_roi_bad_batch_index(lib):
+    """Regions naming no image (batch index -1, B, 7.5 or NaN) pool to zeros;
+    the other regions still equal the brute-force sum over every grid point."""
+    P, S, scale, gamma = (3, 2), 2, 0.5, 0.3
+    x, rois, off = roi_case(85, B=2, P=P, scale=scale, margin=-1.0, off_std=1.0)
+    bad = {1: -1.0, 2: 2.0, 3: 7.5, 4: float("nan")}
+    for n, v in bad.items():
+        rois[n, 0] = v
+    out = oracle.roi_pool_forward(x, rois, off, pooled=P, sampling=S, spatial_scale=scale, gamma=gamma, lib=lib)
+    assert np.all(out[list(bad)] == 0.0), "roi bad batch index"
+    good = [n for n in range(rois.shape[0]) if n not in bad]
+    py, px = roi_positions32(rois[good], off[good], P, S, scale, gamma)
+    B, H, W, C = x.shape
+    gy = np.maximum(0, 1 - np.abs(np.arange(H) - py[..., None]))
+    gx = np.maximum(0, 1 - np.abs(np.arange(W) - px[..., None]))
+    xb = x[rois[good, 0].astype(int)]
+    ref = np.einsum("nijabh,nijabw,nhwc->nijc", gy, gx, xb) / (S * S)
+    assert np.allclose(out[good], ref, rtol=0, atol=1e-12), "roi bad batch index, other regions"
+
+
 def pin_roi_affine(lib):
     """On x = a + b*y + c*x the pooled value is the field at the mean sample position."""
     rng = np.random.default_rng(90)
@@ -572,7 +592,7 @@ def pin_roi_torchvision(lib):
     assert np.allclose(out, ref.permute(0, 2, 3, 1).numpy(), rtol=0, atol=1e-5), "roi torchvision"
 
 
-ROI_PINS = [pin_roi_brute_force, pin_roi_affine, pin_roi_constant, pin_roi_torchvision]
+ROI_PINS = [pin_roi_brute_force, pin_roi_bad_batch_index, pin_roi_affine, pin_roi_constant, pin_roi_torchvision]
 ALL_PINS = ALL_PINS + ROI_PINS
 
 
