@@ -396,10 +396,8 @@ def measure_rows(dcn, dev, stream, l2, barrier, world, steps=280):
         core_fwd(n)
 
     # DCNv3 softmax-mode backward, bf16, at the P3 shape
-    shape, inp = si.workload_core("dcnv3_p3")
-    g = torch.from_numpy(__import__("numpy").random.default_rng(6).standard_normal(
-        (shape.B, shape.Ho, shape.Wo, shape.G * shape.C))).to(torch.bfloat16)
-    t = [inp[k].to(dev) for k in ("x", "offset", "mask")] + [g.to(dev)]
+    shape, inp = si.workload_core("dcnv3_p3_bwd")
+    t = [inp[k].to(dev) for k in ("x", "offset", "mask", "grad_out")]
     R = max(2, math.ceil(4 * l2 / shape.compulsory_bytes(backward=True)))
     sets = [[u.clone() for u in t] + [torch.empty_like(t[0]), torch.empty_like(t[1]), torch.empty_like(t[2])]
             for _ in range(R)]

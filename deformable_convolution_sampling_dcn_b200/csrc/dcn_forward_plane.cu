@@ -17,8 +17,14 @@ namespace dcnb {
 __device__ unsigned int g_device_error = 0;
 
 cudaError_t take_device_error(unsigned int *value) {
+    // The symbol copies below run on the legacy default stream, which does not
+    // wait for work on non-blocking streams (torch's pool streams are such):
+    // without a device-wide synchronisation the read could miss the bit of a
+    // kernel still running there, and the clear could wipe it.
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return e;
     unsigned int zero = 0;
-    cudaError_t e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(unsigned int));
+    e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(unsigned int));
     if (e != cudaSuccess) return e;
     return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned int));
 }

@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(kStagedMaxThreads, 1)
         r_ok = sg.i0 < sg.i1 && it < sg.i1;
         if (!r_ok) return;
         // pixel index inside the segment's (b, g) plane
-        const int lp = (int)(it - (long long)(sg.b * a.G + sg.g) * hw);
+        const int lp = (int)(it - ((long long)sg.b * a.G + sg.g) * hw);
         unsigned wo_u;
         r_ho = (int)fdiv((unsigned)lp, s.fd_wo, wo_u);
         r_wo = (int)wo_u;
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kStagedMaxThreads, 1)
         const uint32_t par = (uint32_t)(n / nbuf) & 1;
         const unsigned char *band = smem + b * buf_bytes;
         const Segment nx = sg.i1 < r1 ? make_segment(sg.i1, r1, s) : Segment{r1, r1, 0, 0, 0, 0, 0};
-        const long long plane_base = (long long)(sg.b * a.G + sg.g) * hw;
+        const long long plane_base = ((long long)sg.b * a.G + sg.g) * hw;
         const long long pix_base = (long long)sg.b * hw;
         const int n_chunks = (int)((sg.i1 - sg.i0 + IPW - 1) / IPW);
         bool ready = false;

@@ -201,6 +201,10 @@ def workload_core(name: str) -> Tuple[CoreShape, Dict[str, torch.Tensor]]:
     if name == "dcnv4_p4_bwd":
         return DCNV4_P4_BWD, core_inputs(DCNV4_P4_BWD, SEEDS[name], offset_std=3.0,
                                          with_grad_out=True)
+    if name == "dcnv3_p3_bwd":
+        # the DCNv3 P3 inputs (same seed and draws) followed by grad_out ~ N(0,1)
+        return DCNV3_P3, core_inputs(DCNV3_P3, SEEDS["dcnv3_p3"], offset_std=4.0, oob_fraction=0.05,
+                                     with_grad_out=True)
     raise KeyError(name)
 
 

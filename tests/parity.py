@@ -4,11 +4,24 @@ The bars (fp32 accumulation in every case):
   fp32 storage:  |gpu - ref| <= 1e-5 * (1 + |ref|)      element by element
   fp16 storage:  |gpu - ref| <= 2e-3 * max|ref|
   bf16 storage:  |gpu - ref| <= 8e-3 * max|ref|
-  atomic backward, fp32:  |gpu - ref| <= 1e-4 * (|ref| + rms(ref))
-The fp16/bf16 bars contain the final rounding of the output to the storage
-type (half an ulp: 2^-11 and 2^-8 relative) plus fp32 summation error.  The
-backward bar is relative to the tensor's own scale because an input
-gradient is a sum of many atomically added contributions that can cancel.
+  backward, fp32 (every gradient):  |gpu - ref| <= 1e-4 * (|ref| + rms(ref))
+  backward, fp16/bf16 grad_offset and grad_mask:
+                 |gpu - ref| <= 2e-3 (fp16) / 8e-3 (bf16) * (|ref| + rms(ref))
+  backward, fp16/bf16 grad_x (packed half-precision atomic adds):
+                 |gpu - ref| <= 2e-2 (fp16) / 1e-1 (bf16) * (|ref| + rms(ref))
+The fp16/bf16 forward bars contain the final rounding of the output to the
+storage type (half an ulp: 2^-11 and 2^-8 relative) plus fp32 summation error.
+"1e-4 relative" for the backward is read per element against the tensor's own
+scale, |ref| + rms(ref): an input gradient is a sum of many atomically added
+contributions that can cancel to far below the size of its terms, so a bar
+on |ref| alone would be meaningless where the sum cancels.
+grad_offset and grad_mask are reduced in fp32 (over the channels of one
+item, by lane shuffles) and stored once: in 16-bit storage their only error
+beyond fp32 summation is that one rounding (at most 2^-11 resp. 2^-8
+relative), which the 2e-3 / 8e-3 bars cover with room to spare while a few
+percent of error (a mis-scaled or dropped term) fails them.  grad_x in
+16-bit storage is summed by packed half-precision atomic adds, each rounding
+to the storage type, so it keeps the wider bars.
 NaN must match NaN exactly.
 """
 from __future__ import annotations
@@ -21,6 +34,8 @@ FWD_TOL = {torch.float32: ("elem", 1e-5), torch.float16: ("max", 2e-3), torch.bf
 # storage type by the GPU, and grad_x is summed by packed half-precision atomic
 # adds (one rounding per addition, up to 4*K*ceil(max tap reach) additions).
 BWD_TOL = {torch.float32: 1e-4, torch.float16: 2e-2, torch.bfloat16: 1e-1}
+# grad_offset / grad_mask: fp32 lane reductions stored once (no atomics).
+BWD_TOL_REDUCED = {torch.float32: 1e-4, torch.float16: 2e-3, torch.bfloat16: 8e-3}
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
@@ -48,14 +63,16 @@ def assert_close_fwd(gpu: torch.Tensor, ref: np.ndarray, what: str = "out") -> f
     return float(ratio.max())
 
 
-def assert_close_bwd(gpu: torch.Tensor, ref: np.ndarray, what: str) -> float:
+def assert_close_bwd(gpu: torch.Tensor, ref: np.ndarray, what: str, atomic: bool = True) -> float:
+    """Backward bar: `atomic` for gradients summed by atomic adds (grad_x),
+    else the tighter bar of gradients reduced in fp32 and stored once."""
     g = to_np(gpu)
     nan_g, nan_r = np.isnan(g), np.isnan(ref)
     assert np.array_equal(nan_g, nan_r), f"{what}: NaN pattern differs"
     g, r = g[~nan_r], ref[~nan_r]
     if r.size == 0:
         return 0.0
-    tol = BWD_TOL[gpu.dtype]
+    tol = (BWD_TOL if atomic else BWD_TOL_REDUCED)[gpu.dtype]
     rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0
     bound = tol * (np.abs(r) + rms)
     err = np.abs(g - r)

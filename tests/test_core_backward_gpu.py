@@ -28,8 +28,8 @@ def run_bwd(shape: si.CoreShape, inp, dev):
 def check_all(got, ref, tag):
     gx, goff, gm = got
     r = [assert_close_bwd(gx, ref["grad_x"], f"{tag} grad_x"),
-         assert_close_bwd(goff, ref["grad_offset"], f"{tag} grad_offset"),
-         assert_close_bwd(gm, ref["grad_mask"], f"{tag} grad_mask")]
+         assert_close_bwd(goff, ref["grad_offset"], f"{tag} grad_offset", atomic=False),
+         assert_close_bwd(gm, ref["grad_mask"], f"{tag} grad_mask", atomic=False)]
     print(f"{tag}: worst err/bound {max(r):.3f}")
 
 
@@ -78,5 +78,14 @@ def test_autograd_function(cuda_dev):
     (out * inp["grad_out"].to(cuda_dev)).sum().backward()
     ref = oracle.dcn_backward(inp["x"], inp["offset"], inp["mask"], inp["grad_out"], G=2)
     assert_close_bwd(x.grad, ref["grad_x"], "autograd grad_x")
-    assert_close_bwd(off.grad, ref["grad_offset"], "autograd grad_offset")
-    assert_close_bwd(m.grad, ref["grad_mask"], "autograd grad_mask")
+    assert_close_bwd(off.grad, ref["grad_offset"], "autograd grad_offset", atomic=False)
+    assert_close_bwd(m.grad, ref["grad_mask"], "autograd grad_mask", atomic=False)
+
+
+def test_dcnv3_p3_softmax_bf16_backward_full_size(cuda_dev):
+    """The DCNv3 P3 backward that bench.py times (bf16, softmax over K, 5 % far
+    taps, 7.4 M taps): at full size the grad_x atomics contend and the softmax
+    Jacobian runs on every (pixel, group)."""
+    shape, inp = si.workload_core("dcnv3_p3_bwd")
+    got, ref = run_bwd(shape, inp, cuda_dev)
+    check_all(got, ref, "dcnv3_p3_bwd")

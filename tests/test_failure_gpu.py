@@ -32,3 +32,17 @@ def test_selftest_rejects_bad_limit(cuda_dev):
 
     with pytest.raises(d.DcnError):
         d._binding.selftest_bounded_wait(0)
+
+
+def test_error_word_seen_from_a_non_blocking_stream(cuda_dev):
+    """A kernel that gives up on a non-blocking stream (torch's side streams are
+    such) must still be reported: reading the word waits for the whole device,
+    not only for the legacy default stream."""
+    import deformable_convolution_sampling_dcn_b200 as d
+
+    assert d._binding.take_device_error() == 0
+    s = torch.cuda.Stream()  # created cudaStreamNonBlocking by torch
+    with torch.cuda.stream(s):
+        d._binding.selftest_bounded_wait(20000)  # 20 ms, no host synchronisation after it
+    assert d._binding.take_device_error() == 1
+    assert d._binding.take_device_error() == 0

@@ -74,8 +74,8 @@ def test_backward(i, cuda_dev):
     torch.cuda.synchronize()
     ref = oracle.dcn_backward(inp["x"], inp["offset"], inp["mask"], inp["grad_out"], G=shape.G, **ogeo(shape))
     assert_close_bwd(gx, ref["grad_x"], f"random grad_x {i}")
-    assert_close_bwd(goff, ref["grad_offset"], f"random grad_offset {i}")
-    assert_close_bwd(gm, ref["grad_mask"], f"random grad_mask {i}")
+    assert_close_bwd(goff, ref["grad_offset"], f"random grad_offset {i}", atomic=False)
+    assert_close_bwd(gm, ref["grad_mask"], f"random grad_mask {i}", atomic=False)
 
 
 def draw_proj(i):
