@@ -473,9 +473,10 @@ def measure_rows(dcn, dev, stream, l2, barrier, world, steps=280):
                        "GB_s": round(rs.compulsory_bytes() / ms / 1e6, 1), "R": R}
     del sets
 
-    # DCNv4 P4 core fused with its 512 -> 512 projection (tensor cores), and for
-    # context the same two steps unfused: the core kernel, then a cuBLAS GEMM
-    # through torch on the stored core output.
+    # DCNv4 P4 core followed by its 512 -> 512 projection (tensor cores): the
+    # workspace route (core kernel into a workspace, then the library's GEMM),
+    # the one fused kernel, and for context the core kernel followed by a
+    # cuBLAS GEMM through torch on the stored core output.
     shape, inp = si.workload_proj()
     t = [inp[k].to(dev) for k in ("x", "offset", "mask", "weight", "bias")]
     cout = t[3].shape[0]
@@ -486,10 +487,16 @@ def measure_rows(dcn, dev, stream, l2, barrier, world, steps=280):
                                       torch.empty((shape.B, shape.Ho, shape.Wo, shape.G * shape.C),
                                                   dtype=t[0].dtype, device=dev)] for _ in range(R)]
 
-    def mkp(s):
-        return lambda: dcn.dcn_core_forward_proj(s[0], s[1], s[2], s[3], s[4], group=shape.G, out=s[5])
+    def mkp(s):  # workspace route; the core-output buffer is its workspace
+        return lambda: dcn.dcn_core_forward_proj(s[0], s[1], s[2], s[3], s[4], group=shape.G, out=s[5],
+                                                 workspace=s[6])
 
     ms = time_steps(mkp, sets, steps, 3 * R, stream, barrier, world) / steps
+
+    def mkf(s):
+        return lambda: dcn.dcn_core_forward_proj(s[0], s[1], s[2], s[3], s[4], group=shape.G, out=s[5], fused=True)
+
+    ms_f = time_steps(mkf, sets, steps, 3 * R, stream, barrier, world) / steps
 
     def mku(s):
         def call():
@@ -501,7 +508,9 @@ def measure_rows(dcn, dev, stream, l2, barrier, world, steps=280):
     flops = 2.0 * shape.B * shape.Ho * shape.Wo * cout * shape.G * shape.C
     out["dcnv4_p4_proj"] = {"us": round(ms * 1e3, 2), "Gsamples_s": round(shape.samples / ms / 1e6, 2),
                             "GB_s": round(pbytes / ms / 1e6, 1), "gemm_TFLOP_s": round(flops / ms / 1e9, 1),
-                            "unfused_core_then_cublas_us": round(ms_u * 1e3, 2), "Cout": cout, "R": R}
+                            "route": "workspace (core kernel + tcgen05 GEMM)", "fused_one_kernel_us":
+                            round(ms_f * 1e3, 2), "unfused_core_then_cublas_us": round(ms_u * 1e3, 2),
+                            "Cout": cout, "R": R}
     del sets
 
     # modulated deformable convolution (a dense weight per kernel point) at the
@@ -676,6 +685,56 @@ def run_case(name: str, calls: int) -> None:
     print(f"ok {name} x{calls}")
 
 
+def run_ceilings(reps_scale: float) -> None:
+    """Measure the on-chip rates that bound the sampling kernels (dcn_probe_rate:
+    one CTA per SM, SM-clock cycles) and print them, per SM per clock, with the
+    lower bound each implies for the DCNv4 P4 forward (1,843,200 samples on all
+    SMs at the maximum SM clock).  One JSON line at the end."""
+    import deformable_convolution_sampling_dcn_b200 as dcn
+
+    dev = torch.device("cuda:0")
+    props = torch.cuda.get_device_properties(dev)
+    sms = props.multi_processor_count
+    clk_mhz = float(_nvml_max_sm_clock() or 1965.0)
+    # repetitions giving a few milliseconds per probe
+    reps = {"lds128": 20000, "chunk_f32_ffma2": 80000, "ffma": 20000, "ffma2": 20000, "chunk_f16_ffma": 80000,
+            "chunk_f16_ffma2": 80000, "chunk_bf16_ffma2": 80000, "chunk_f16_mixed": 80000,
+            "ldg128_l1": 20000, "gather4": 2000, "gather8": 2000, "gather8_ffma": 2000, "alu": 20000}
+    res = {}
+    for name in dcn._binding.PROBES:
+        n = max(1, int(reps[name] * reps_scale))
+        dcn._binding.probe_rate(name, max(1, n // 10))  # warm-up
+        best, unit = 0.0, ""
+        for _ in range(3):
+            r, unit = dcn._binding.probe_rate(name, n)
+            best = max(best, r)
+        res[name] = {"per_sm_per_clk": round(best, 4), "unit": unit}
+    samples = si.DCNV4_P4.samples
+    for name in ("gather4", "gather8", "gather8_ffma"):
+        r = res[name]["per_sm_per_clk"]
+        res[name]["p4_floor_us"] = round(samples / (sms * r * clk_mhz * 1e6) * 1e6, 2)
+    # smem-data floor of any design that reads every corner row from shared memory or L1 once per tap
+    lds = res["lds128"]["per_sm_per_clk"]
+    tap_bytes = samples * 4 * si.DCNV4_P4.C * 2
+    res["p4_corner_bytes_floor_us"] = round(tap_bytes / (sms * lds * clk_mhz * 1e6) * 1e6, 2)
+    for name, v in res.items():
+        if isinstance(v, dict):
+            extra = f"   P4 floor {v['p4_floor_us']} us" if "p4_floor_us" in v else ""
+            print(f"{name:18s} {v['per_sm_per_clk']:10.3f} {v['unit']}/SM/clk{extra}")
+    print(json.dumps({"ceilings": res, "sms": sms, "sm_max_mhz": clk_mhz}))
+
+
+def _nvml_max_sm_clock():
+    try:
+        import pynvml
+
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(torch.cuda.current_device())
+        return pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+    except Exception:
+        return None
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -688,7 +747,13 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--case", choices=CASES, default=None,
                     help="only call this workload's entry point --steps times, untimed (for profilers)")
+    ap.add_argument("--ceilings", action="store_true",
+                    help="only measure the on-chip rate probes (shared loads, conversions, FMAs, gather loops)")
+    ap.add_argument("--ceilings-scale", type=float, default=1.0, help="scale of the probes' repetition counts")
     args = ap.parse_args()
+    if args.ceilings:
+        run_ceilings(args.ceilings_scale)
+        return
     if args.case is not None:
         run_case(args.case, args.steps)
         return

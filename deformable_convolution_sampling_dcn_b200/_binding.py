@@ -27,8 +27,9 @@ _DTYPE_CODE = {torch.float32: DCN_F32, torch.float16: DCN_F16, torch.bfloat16: D
 EXPORTS = ("dcn_core_output_hw", "dcn_core_forward", "dcn_core_backward", "deform_agg_forward",
            "deform_agg_backward", "dcn_status_string", "dcn_last_error_detail", "dcn_abi_version",
            "dcn_take_device_error", "deform_roi_pool_forward", "dcn_core_forward_proj",
-           "dcn_selftest_bounded_wait", "dcn_deform_conv_forward")
-ABI_VERSION = 1
+           "dcn_selftest_bounded_wait", "dcn_deform_conv_forward", "dcn_probe_rate",
+           "dcn_core_forward_proj_workspace_bytes")
+ABI_VERSION = 2
 
 
 class DcnParams(ctypes.Structure):
@@ -79,14 +80,19 @@ def _declare(lib):
     lib.dcn_abi_version.restype = ctypes.c_int32
     lib.deform_roi_pool_forward.argtypes = [ctypes.POINTER(DroiParams), vp, vp, vp, vp, vp]
     lib.deform_roi_pool_forward.restype = st
-    lib.dcn_core_forward_proj.argtypes = [P, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp]
+    lib.dcn_core_forward_proj.argtypes = [P, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int64, vp]
     lib.dcn_core_forward_proj.restype = st
+    lib.dcn_core_forward_proj_workspace_bytes.argtypes = [P]
+    lib.dcn_core_forward_proj_workspace_bytes.restype = ctypes.c_int64
     lib.dcn_deform_conv_forward.argtypes = [P, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp]
     lib.dcn_deform_conv_forward.restype = st
     lib.dcn_selftest_bounded_wait.argtypes = [ctypes.c_int32, vp]
     lib.dcn_selftest_bounded_wait.restype = st
     lib.dcn_take_device_error.argtypes = []
     lib.dcn_take_device_error.restype = ctypes.c_int32
+    lib.dcn_probe_rate.argtypes = [ctypes.c_int32, ctypes.c_int32, vp, ctypes.c_int64,
+                                   ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_char_p), vp]
+    lib.dcn_probe_rate.restype = st
     return lib
 
 
@@ -155,6 +161,23 @@ def take_device_error() -> int:
     return int(lib().dcn_take_device_error())
 
 
+PROBES = ("lds128", "chunk_f32_ffma2", "ffma", "ffma2", "chunk_f16_ffma", "chunk_f16_ffma2", "chunk_bf16_ffma2",
+          "chunk_f16_mixed", "ldg128_l1", "gather4", "gather8", "gather8_ffma", "alu")
+
+
+def probe_rate(name: str, reps: int, device=None) -> Tuple[float, str]:
+    """Run one on-chip rate probe; returns (units per SM per clock, unit)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    buf = torch.zeros(65536, dtype=torch.uint8, device=dev)
+    units = ctypes.c_double()
+    unit = ctypes.c_char_p()
+    check(lib().dcn_probe_rate(PROBES.index(name), int(reps), buf.data_ptr(), buf.numel(), ctypes.byref(units),
+                               ctypes.byref(unit), torch.cuda.current_stream(dev).cuda_stream))
+    torch.cuda.synchronize(dev)
+    words = buf[:16].view(torch.int64).cpu().tolist()
+    return units.value * words[1] / words[0], unit.value.decode()
+
+
 def selftest_bounded_wait(limit_us: int = 2000, device=None) -> None:
     """Enqueue the bounded-wait self-test on the current stream (see dcn_b200.h)."""
     check(lib().dcn_selftest_bounded_wait(int(limit_us), torch.cuda.current_stream(device).cuda_stream))
@@ -194,8 +217,13 @@ def dcn_core_forward(x: torch.Tensor, offset: torch.Tensor, mask: torch.Tensor, 
 def dcn_core_forward_proj(x: torch.Tensor, offset: torch.Tensor, mask: torch.Tensor, weight: torch.Tensor,
                           bias: Optional[torch.Tensor] = None, *, group: int, kernel=(3, 3), stride=(1, 1),
                           pad=(1, 1), dil=(1, 1), offset_scale: float = 1.0, softmax: bool = False,
-                          out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """out [B,Ho,Wo,Cout] = bias + core(x, offset, mask) . weight[Cout, G*C]^T in one kernel; see dcn_b200.h."""
+                          out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                          fused: bool = False) -> torch.Tensor:
+    """out [B,Ho,Wo,Cout] = bias + core(x, offset, mask) . weight[Cout, G*C]^T; see dcn_b200.h.
+
+    By default the core goes through a workspace (`workspace`, or one torch
+    allocates here) and a tensor-core GEMM projects it; fused=True runs the one
+    fused kernel with no workspace."""
     _cuda_tensor("x", x)
     p = core_params(x, group, kernel, stride, pad, dil, offset_scale, softmax)
     Ho, Wo = dcn_core_output_hw(p)
@@ -220,9 +248,17 @@ def dcn_core_forward_proj(x: torch.Tensor, offset: torch.Tensor, mask: torch.Ten
         _cuda_tensor("out", out, x.dtype)
         if tuple(out.shape) != (p.B, Ho, Wo, cout):
             raise ValueError("out has the wrong shape")
+    ws_ptr, ws_bytes = None, 0
+    if not fused:
+        need = int(lib().dcn_core_forward_proj_workspace_bytes(ctypes.byref(p)))
+        if workspace is None:
+            workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+        else:
+            _cuda_tensor("workspace", workspace)
+        ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     check(lib().dcn_core_forward_proj(ctypes.byref(p), cout, x.data_ptr(), offset.data_ptr(), mask.data_ptr(),
                                       weight.data_ptr(), None if bias is None else bias.data_ptr(),
-                                      out.data_ptr(), _stream(x)))
+                                      out.data_ptr(), ws_ptr, ws_bytes, _stream(x)))
     return out
 
 

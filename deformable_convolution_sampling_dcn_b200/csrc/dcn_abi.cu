@@ -164,9 +164,16 @@ dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offs
 
 namespace {
 
+// Bytes of the core output [B, Ho, Wo, G*C] (-1 for invalid params).
+long long core_out_bytes(const dcn_params *p) {
+    int Ho = 0, Wo = 0;
+    if (check_core(p, &Ho, &Wo) != DCN_OK) return -1;
+    return (long long)p->B * Ho * Wo * p->G * p->C * (long long)dtype_size(p->dtype);
+}
+
 dcn_status proj_call(const dcn_params *p, int32_t Cout, const void *x, const void *offset, const void *mask,
-                     const void *weight, const void *bias, void *out, dcn_stream_t stream, bool per_point,
-                     const char *what) {
+                     const void *weight, const void *bias, void *out, void *workspace, int64_t workspace_bytes,
+                     dcn_stream_t stream, bool per_point, const char *what) {
     int Ho = 0, Wo = 0;
     dcn_status s = check_core(p, &Ho, &Wo);
     if (s != DCN_OK) return s;
@@ -189,6 +196,21 @@ dcn_status proj_call(const dcn_params *p, int32_t Cout, const void *x, const voi
         return fail(DCN_ERR_ALIGN, "x, weight and out must be 16-byte aligned");
     if (!aligned(offset, 4) || !aligned(mask, 2) || !aligned(bias, 2))
         return fail(DCN_ERR_ALIGN, "offset must be 4-byte aligned, mask and bias 2-byte aligned");
+    const long long need = core_out_bytes(p);
+    if (!per_point && workspace && workspace_bytes >= need) {
+        // two launches: the core into the workspace (staged kernel where it applies),
+        // then the tensor-core projection of that [B*Ho*Wo, G*C] matrix
+        if (!aligned(workspace, 16)) return fail(DCN_ERR_ALIGN, "workspace must be 16-byte aligned");
+        dcnb::CoreArgs c = core_args(p, Ho, Wo);
+        c.x = x; c.offset = offset; c.mask = mask; c.out = workspace;
+        bool handled = false;
+        cudaError_t e = dcnb::launch_core_forward_plane(c, (cudaStream_t)stream, &handled);
+        if (e == cudaSuccess && !handled) e = dcnb::launch_core_forward_generic(c, (cudaStream_t)stream);
+        if (e == cudaSuccess)
+            e = dcnb::launch_proj_gemm(workspace, weight, bias, out, (long long)p->B * Ho * Wo, (int)GC, Cout,
+                                       (dcnb::DType)p->dtype, (cudaStream_t)stream);
+        return cuda_status(e, what);
+    }
     dcnb::ProjArgs a;
     a.core = core_args(p, Ho, Wo);
     a.core.x = x; a.core.offset = offset; a.core.mask = mask; a.core.out = out;
@@ -203,14 +225,23 @@ dcn_status proj_call(const dcn_params *p, int32_t Cout, const void *x, const voi
 
 dcn_status dcn_core_forward_proj(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
                                  const void *mask, const void *weight, const void *bias, void *out,
-                                 dcn_stream_t stream) {
-    return proj_call(p, Cout, x, offset, mask, weight, bias, out, stream, false, "dcn_core_forward_proj launch");
+                                 void *workspace, int64_t workspace_bytes, dcn_stream_t stream) {
+    if (workspace_bytes < 0) return fail(DCN_ERR_SHAPE, "workspace_bytes is negative");
+    return proj_call(p, Cout, x, offset, mask, weight, bias, out, workspace, workspace_bytes, stream, false,
+                     "dcn_core_forward_proj launch");
+}
+
+int64_t dcn_core_forward_proj_workspace_bytes(const dcn_params *p) {
+    const long long n = core_out_bytes(p);
+    if (n < 0) fail(DCN_ERR_SHAPE, "invalid params");
+    return n;
 }
 
 dcn_status dcn_deform_conv_forward(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
                                    const void *mask, const void *weight, const void *bias, void *out,
                                    dcn_stream_t stream) {
-    return proj_call(p, Cout, x, offset, mask, weight, bias, out, stream, true, "dcn_deform_conv_forward launch");
+    return proj_call(p, Cout, x, offset, mask, weight, bias, out, nullptr, 0, stream, true,
+                     "dcn_deform_conv_forward launch");
 }
 
 dcn_status dcn_core_backward(const dcn_params *p, const void *x, const void *offset, const void *mask,

@@ -75,6 +75,10 @@ cudaError_t take_device_error(unsigned int *value);
 cudaError_t launch_bounded_wait_selftest(long long limit_ns, cudaStream_t stream);
 // Fused core + projection (tcgen05 GEMM on the core tile in shared memory).
 cudaError_t launch_core_forward_proj(const ProjArgs &a, cudaStream_t stream);
+// out[p, o] = bias[o] + sum_j core[p, j] * weight[o, j] on the tensor cores (fp16/bf16;
+// core [P, KD], weight [Cout, KD], out [P, Cout]; KD a multiple of 64, Cout of 8 up to 512).
+cudaError_t launch_proj_gemm(const void *core, const void *weight, const void *bias, void *out, long long P, int KD,
+                             int Cout, DType dtype, cudaStream_t stream);
 cudaError_t launch_agg_forward(const AggArgs &a, cudaStream_t stream);
 // Anchor-wide aggregation kernels (all groups per CTA); sets *handled = false
 // (and launches nothing) when the feature row width does not fit them.

@@ -1,0 +1,374 @@
+// On-chip rate probes: measurement support for the roofline of the sampling
+// kernels (no counterpart on the pages).  Each probe runs one CTA of 512
+// threads per SM (its shared-memory request allows no second one), times its
+// loop with the SM clock and adds the cycles to a caller-owned device word,
+// so the host gets a rate per SM per clock that does not depend on the clock
+// speed.  Every shared-memory load is a volatile one and every arithmetic
+// probe feeds on data loaded in the same repetition or on a loop-carried
+// accumulator, so the assembler can neither hoist nor merge the measured
+// instructions; the chunk probes read one 16-byte chunk of channels per
+// repetition (one shared load) and widen and accumulate it, the way a gather
+// does per corner row; the gather probes replay the inner loop of a sampling
+// kernel over records and a band of random 16-bit values laid out as the
+// staged kernel lays them out.
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "dcn_b200.h"
+
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kSmem = 128 * 1024;      // one CTA per SM; band + records of the gather probes
+constexpr int kBandRows = 36;          // band of the DCNv4 P4 staged kernel: 36 rows of
+constexpr int kBandCols = 42;          //   W + 2 = 42 pixels of 64 bytes (fp16, C = 32)
+constexpr int kRowBytes = kBandCols * 64;
+constexpr int kBandBytes = kBandRows * kRowBytes;  // 96,768 bytes
+constexpr int kRecs = 8;               // records per item slot, cycled through
+constexpr int kL1Bytes = 32 * 1024;    // L1-resident source of the global-load probe
+
+enum Probe : int {
+    kLds128 = 0,        // 16-byte shared loads, each quarter warp one 128-byte line
+    kChunkF32Ffma2 = 1, // two 16-byte loads of 4 fp32 each + 4 paired FMAs (8 channels of an fp32 row)
+    kFfma = 2,          // fma.rn.f32
+    kFfma2 = 3,         // fma.rn.f32x2 (two FMAs)
+    kChunkF16Ffma = 4,  // 16-byte load + 8 fp16 -> fp32 conversions + 8 scalar FMAs (one chunk)
+    kChunkF16Ffma2 = 5, // load + 8 conversions + 4 paired FMAs
+    kChunkBf16Ffma2 = 6,// load + bf16 widening by shift/mask (8 ALU ops) + 4 paired FMAs
+    kChunkF16Mixed = 7, // load + 8 fma.rn.f32.f16 (fp16 operands, fp32 accumulator)
+    kLdg128L1 = 8,      // 16-byte global loads that hit L1
+    kGather4 = 9,       // 4 lanes per 64-byte item, 4 loads per tap (corner rows A, B apart)
+    kGather8 = 10,      // 8 lanes per item, 2 loads per tap (A|B as one 128-byte row), paired FMAs
+    kGather8Ffma = 11,  // as kGather8 with scalar FMAs
+    kAlu = 12,          // lop3.b32 (integer pipe)
+    kNumProbes = 13
+};
+
+// Work units per thread per repetition, and their name.
+__host__ __device__ constexpr double units_per_rep(int p) {
+    return p == kLds128 ? 8.0 * 16.0          // bytes
+         : p == kChunkF32Ffma2 ? 1.0          // chunks (8 channels)
+         : p == kFfma ? 16.0                  // FMAs
+         : p == kFfma2 ? 16.0                 // FMAs (8 instructions)
+         : p <= kChunkF16Mixed ? 1.0          // chunks (8 channels of one corner)
+         : p == kLdg128L1 ? 8.0 * 16.0        // bytes
+         : p == kGather4 ? 9.0 / 4.0          // samples (9 taps, 4 lanes per item)
+         : p <= kGather8Ffma ? 9.0 / 8.0      // samples (9 taps, 8 lanes per item)
+         : 16.0;                              // ALU ops
+}
+
+const char *unit_name(int p) {
+    switch (p) {
+        case kLds128: case kLdg128L1: return "bytes";
+        case kFfma: case kFfma2: return "fma";
+        case kGather4: case kGather8: case kGather8Ffma: return "samples";
+        case kAlu: return "alu ops";
+        default: return "chunks";
+    }
+}
+
+__device__ __forceinline__ uint32_t hash32(uint32_t x) {
+    x ^= x >> 16;
+    x *= 0x7feb352du;
+    x ^= x >> 15;
+    x *= 0x846ca68bu;
+    x ^= x >> 16;
+    return x;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.volatile.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.volatile.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+
+// Two fp16 of a word -> an fp32 pair in one 64-bit register.
+__device__ __forceinline__ uint64_t cvt2(uint32_t h) {
+    uint64_t v;
+    asm volatile("{.reg .f16 lo, hi; .reg .f32 a, b;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 a, lo;\n\t"
+                 "cvt.f32.f16 b, hi;\n\tmov.b64 %0, {a, b};}" : "=l"(v) : "r"(h));
+    return v;
+}
+__device__ __forceinline__ void ffma2(uint64_t &acc, uint64_t w, uint64_t v) {
+    asm volatile("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(w), "l"(v));
+}
+__device__ __forceinline__ void ffma(float &acc, float w, float v) {
+    asm volatile("fma.rn.f32 %0, %1, %2, %0;" : "+f"(acc) : "f"(w), "f"(v));
+}
+__device__ __forceinline__ uint64_t pack2(float a, float b) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(a), "f"(b));
+    return v;
+}
+__device__ __forceinline__ float2 unpack2(uint64_t v) {
+    float2 f;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
+    return f;
+}
+
+template <int P>
+__global__ void __launch_bounds__(kThreads, 1)
+    probe_kernel(int reps, unsigned long long *res, const uint4 *gsrc) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+    uint32_t sink = 0;
+
+    // fill the band with random fp16 in [-1, 1) and build each warp's records
+    for (int i = threadIdx.x; i < kBandBytes / 4; i += kThreads) {
+        const uint32_t r = hash32(i * 2654435761u + blockIdx.x);
+        const __half2 h = __floats2half2_rn((float)(r & 0xffff) / 32768.0f - 1.0f, (float)(r >> 16) / 32768.0f - 1.0f);
+        reinterpret_cast<__half2 *>(smem)[i] = h;
+    }
+    // records: kRecs per item slot of the warp, 32 bytes each, after the band
+    unsigned char *recs = smem + kBandBytes + warp * (kRecs * 8 * 32);
+    for (int i = lane; i < kRecs * 8; i += 32) {
+        const uint32_t r = hash32(0x9e3779b9u * (uint32_t)(warp * kRecs * 8 + i) + blockIdx.x * 7919u);
+        const int y = (int)(r % (kBandRows - 1)), x = (int)((r >> 8) % (kBandCols - 1));
+        const int Pa = (y * kBandCols + x) * 64;
+        const float w0 = 0.25f + (float)(r & 7) * 0.01f, w1 = 0.5f - w0;
+        if (P == kGather4) {
+            // point-major [rec][item slot 0..7]: weights float4, then addresses (A, B) in the order
+            // that puts the two 64-byte reads of a quarter warp into different bank halves
+            const int slot = i & 7;
+            const bool order = ((Pa >> 6) ^ slot) & 1;
+            reinterpret_cast<float4 *>(recs)[i] = make_float4(w0, w1, w1, w0);
+            reinterpret_cast<int2 *>(recs + kRecs * 8 * 16)[i] = order ? make_int2(Pa + 64, Pa) : make_int2(Pa, Pa + 64);
+        } else {
+            // [rec][item slot 0..3][half]: {P, w_top, w_bottom, 0} for corner A, then for corner B
+            reinterpret_cast<float4 *>(recs)[2 * i] = make_float4(__int_as_float(Pa), w0, w1, 0.0f);
+            reinterpret_cast<float4 *>(recs)[2 * i + 1] = make_float4(__int_as_float(Pa), w1, w0, 0.0f);
+        }
+    }
+    __syncthreads();
+    const uint32_t rbase = (uint32_t)__cvta_generic_to_shared(recs);
+    long long t0 = clock64();
+
+    if (P == kLds128) {
+        uint32_t a = sbase + (uint32_t)(warp * 512 + lane * 16);
+        for (int r = 0; r < reps; ++r) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const uint4 v = lds128(a + j * 8192);
+                sink ^= v.x ^ v.w;
+            }
+            a ^= 4096;
+        }
+    } else if (P == kFfma || P == kFfma2) {
+        uint64_t acc2[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        const uint64_t w = pack2(0.5f, 0.5f);
+        for (int r = 0; r < reps; ++r) {
+            if (P == kFfma) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) ffma(acc[j & 7], 0.5f, 0.25f);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) ffma2(acc2[j], w, w);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sink ^= __float_as_uint(acc[j]) ^ (uint32_t)acc2[j];
+    } else if ((P >= kChunkF16Ffma && P <= kChunkF16Mixed) || P == kChunkF32Ffma2) {
+        // one 16-byte chunk per repetition from a rotating, conflict-free position
+        uint32_t a = sbase + (uint32_t)(warp * 2048 + lane * 16);
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        uint64_t acc2[4] = {0, 0, 0, 0};
+        const uint64_t w = pack2(0.5f, 0.25f);
+        const uint32_t wh = 0x38003400u;  // (0.5, 0.25) in fp16
+        for (int r = 0; r < reps; ++r) {
+            const uint4 v = lds128(a);
+            const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+            if (P == kChunkF16Ffma) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = unpack2(cvt2(h[j]));
+                    ffma(acc[2 * j], 0.5f, f.x);
+                    ffma(acc[2 * j + 1], 0.5f, f.y);
+                }
+            } else if (P == kChunkF16Ffma2) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) ffma2(acc2[j], w, cvt2(h[j]));
+            } else if (P == kChunkBf16Ffma2) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t lo, hi;
+                    asm volatile("shl.b32 %0, %1, 16;" : "=r"(lo) : "r"(h[j]));
+                    asm volatile("and.b32 %0, %1, 0xffff0000;" : "=r"(hi) : "r"(h[j]));
+                    ffma2(acc2[j], w, pack2(__uint_as_float(lo), __uint_as_float(hi)));
+                }
+            } else if (P == kChunkF16Mixed) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    asm volatile("{.reg .f16 a0, a1, w0, w1;\n\tmov.b32 {a0, a1}, %2;\n\tmov.b32 {w0, w1}, %3;\n\t"
+                                 "fma.rn.f32.f16 %0, a0, w0, %0;\n\tfma.rn.f32.f16 %1, a1, w1, %1;}"
+                                 : "+f"(acc[2 * j]), "+f"(acc[2 * j + 1]) : "r"(h[j]), "r"(wh));
+            } else {  // fp32 row: 8 channels in two 16-byte loads
+                const uint4 v2 = lds128(a + 16);
+                ffma2(acc2[0], w, ((uint64_t)v.y << 32) | v.x);
+                ffma2(acc2[1], w, ((uint64_t)v.w << 32) | v.z);
+                ffma2(acc2[2], w, ((uint64_t)v2.y << 32) | v2.x);
+                ffma2(acc2[3], w, ((uint64_t)v2.w << 32) | v2.z);
+            }
+            a ^= (uint32_t)(((r & 3) + 1) * 512);  // next chunk: another 512-byte line of this warp's 2 KB
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sink ^= __float_as_uint(acc[j]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sink ^= (uint32_t)acc2[j];
+    } else if (P == kLdg128L1) {
+        const unsigned char *src = reinterpret_cast<const unsigned char *>(gsrc);
+        uint32_t o = (uint32_t)(threadIdx.x * 16) & (kL1Bytes - 1);
+        for (int r = 0; r < reps; ++r) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint4 v;
+                asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                             : "l"(src + ((o + j * 4096) & (kL1Bytes - 1))));
+                sink ^= v.x ^ v.w;
+            }
+            o += 512;
+        }
+    } else if (P == kGather4) {
+        const int gi = lane >> 2, q = lane & 3;
+        const uint32_t bq = sbase + q * 16;
+        const uint32_t rw = rbase + gi * 16, ra = rbase + kRecs * 8 * 16 + gi * 8;
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        int rec = 0;
+        for (int r = 0; r < reps; ++r) {
+#pragma unroll
+            for (int k = 0; k < 9; ++k) {
+                const uint4 wr = lds128(rw + rec * 128);
+                const uint2 ad = lds64(ra + rec * 64);
+                const float w[4] = {__uint_as_float(wr.x), __uint_as_float(wr.y), __uint_as_float(wr.z),
+                                    __uint_as_float(wr.w)};
+                const uint4 v[4] = {lds128(bq + ad.x), lds128(bq + ad.x + kRowBytes), lds128(bq + ad.y),
+                                    lds128(bq + ad.y + kRowBytes)};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t hw[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f = unpack2(cvt2(hw[j]));
+                        ffma(acc[2 * j], w[c], f.x);
+                        ffma(acc[2 * j + 1], w[c], f.y);
+                    }
+                }
+                rec = (rec + 1) & (kRecs - 1);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sink ^= __float_as_uint(acc[j]);
+    } else if (P == kGather8 || P == kGather8Ffma) {
+        const int gi = lane >> 3, q = lane & 7;
+        const uint32_t bq = sbase + q * 16;
+        const uint32_t rr = rbase + gi * 32 + (q >> 2) * 16;
+        uint64_t acc2[4] = {0, 0, 0, 0};
+        float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        int rec = 0;
+        for (int r = 0; r < reps; ++r) {
+#pragma unroll
+            for (int k = 0; k < 9; ++k) {
+                const uint4 rc = lds128(rr + rec * 128);
+                const uint32_t a = bq + rc.x;
+                const uint4 top = lds128(a), bot = lds128(a + kRowBytes);
+                const uint32_t t[4] = {top.x, top.y, top.z, top.w}, b[4] = {bot.x, bot.y, bot.z, bot.w};
+                if (P == kGather8) {
+                    const uint64_t wt = pack2(__uint_as_float(rc.y), __uint_as_float(rc.y));
+                    const uint64_t wb = pack2(__uint_as_float(rc.z), __uint_as_float(rc.z));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        ffma2(acc2[j], wt, cvt2(t[j]));
+                        ffma2(acc2[j], wb, cvt2(b[j]));
+                    }
+                } else {
+                    const float wt = __uint_as_float(rc.y), wb = __uint_as_float(rc.z);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 ft = unpack2(cvt2(t[j])), fb = unpack2(cvt2(b[j]));
+                        ffma(acc[2 * j], wt, ft.x);
+                        ffma(acc[2 * j + 1], wt, ft.y);
+                        ffma(acc[2 * j], wb, fb.x);
+                        ffma(acc[2 * j + 1], wb, fb.y);
+                    }
+                }
+                rec = (rec + 1) & (kRecs - 1);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sink ^= (uint32_t)acc2[j];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sink ^= __float_as_uint(acc[j]);
+    } else if (P == kAlu) {
+        uint32_t v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = lane * 8 + j;
+        for (int r = 0; r < reps; ++r) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                asm volatile("lop3.b32 %0, %0, %1, %2, 0x96;" : "+r"(v[j & 7]) : "r"(j), "r"(r));
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sink ^= v[j];
+    }
+
+    __syncthreads();
+    const long long t1 = clock64();
+    if (threadIdx.x == 0) {
+        atomicAdd(res + 0, (unsigned long long)(t1 - t0));
+        atomicAdd(res + 1, 1ull);
+    }
+    if (sink == 0x12345678u) atomicAdd(res + 2, 1ull);  // keeps every result live
+}
+
+template <int P>
+cudaError_t launch_probe(int reps, int sms, unsigned long long *res, const uint4 *src, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(probe_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    probe_kernel<P><<<sms, kThreads, kSmem, st>>>(reps, res, src);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" dcn_status dcn_probe_rate(int32_t probe, int32_t reps, void *dev_buf, int64_t dev_buf_bytes,
+                                     double *units_per_cta, const char **unit, dcn_stream_t stream) {
+    if (!dev_buf || !units_per_cta || !unit) return DCN_ERR_NULL;
+    if (probe < 0 || probe >= kNumProbes || reps < 1 || reps > (1 << 24)) return DCN_ERR_SHAPE;
+    if (dev_buf_bytes < 4096 + kL1Bytes) return DCN_ERR_SHAPE;
+    if (reinterpret_cast<uintptr_t>(dev_buf) % 256 != 0) return DCN_ERR_ALIGN;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DCN_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    unsigned long long *res = static_cast<unsigned long long *>(dev_buf);
+    if (cudaMemsetAsync(res, 0, 3 * sizeof(unsigned long long), st) != cudaSuccess) return DCN_ERR_CUDA;
+    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<unsigned char *>(dev_buf) + 4096);
+    cudaError_t e = cudaErrorInvalidValue;
+    switch (probe) {
+        case kLds128: e = launch_probe<kLds128>(reps, sms, res, src, st); break;
+        case kChunkF32Ffma2: e = launch_probe<kChunkF32Ffma2>(reps, sms, res, src, st); break;
+        case kFfma: e = launch_probe<kFfma>(reps, sms, res, src, st); break;
+        case kFfma2: e = launch_probe<kFfma2>(reps, sms, res, src, st); break;
+        case kChunkF16Ffma: e = launch_probe<kChunkF16Ffma>(reps, sms, res, src, st); break;
+        case kChunkF16Ffma2: e = launch_probe<kChunkF16Ffma2>(reps, sms, res, src, st); break;
+        case kChunkBf16Ffma2: e = launch_probe<kChunkBf16Ffma2>(reps, sms, res, src, st); break;
+        case kChunkF16Mixed: e = launch_probe<kChunkF16Mixed>(reps, sms, res, src, st); break;
+        case kLdg128L1: e = launch_probe<kLdg128L1>(reps, sms, res, src, st); break;
+        case kGather4: e = launch_probe<kGather4>(reps, sms, res, src, st); break;
+        case kGather8: e = launch_probe<kGather8>(reps, sms, res, src, st); break;
+        case kGather8Ffma: e = launch_probe<kGather8Ffma>(reps, sms, res, src, st); break;
+        case kAlu: e = launch_probe<kAlu>(reps, sms, res, src, st); break;
+    }
+    if (e != cudaSuccess) return DCN_ERR_CUDA;
+    *units_per_cta = units_per_rep(probe) * (double)kThreads * (double)reps;
+    *unit = unit_name(probe);
+    return DCN_OK;
+}

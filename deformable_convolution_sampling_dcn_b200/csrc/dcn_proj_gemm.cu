@@ -1,0 +1,287 @@
+// Pointwise projection on the tensor cores (sm_100a): the 1x1 convolution
+// with bias that follows the sampling core in the DCNv4 module (YOLOv11 +
+// DCNv4 page, section 3.2, proj_conv), as a plain GEMM over a core output
+// that already sits in device memory:
+//   out[p, o] = bias[o] + sum_j core[p, j] * weight[o, j]
+// core [P, KD] and weight [Cout, KD] are both K-major (row-major with the
+// contraction index fastest), fp16 or bf16; out [P, Cout] in the same type.
+//
+// Persistent, warp-specialised: warp 0 streams (pixel tile, weight tile)
+// K-blocks of 64 channels by TMA (128-byte swizzle) through a 4-stage ring,
+// one thread of warp 1 issues tcgen05.mma (M = 128 pixels, N = up to 256
+// output channels, K = 16) into one of two tensor-memory accumulators, and
+// warps 2..5 (one per 32-lane quarter of tensor memory) read the finished
+// accumulator back with tcgen05.ld, add the bias in fp32, round once to the
+// storage type and store, while the products of the next tile already run
+// into the other accumulator.  Every wait is bounded and gives up when
+// another role has aborted; a role that gives up sets the device error word.
+#include <cudaTypedefs.h>
+
+#include <type_traits>
+
+#include "dcn_common.cuh"
+#include "dcn_device.h"
+#include "dcn_launch.h"
+#include "dcn_tcgen05.cuh"
+
+namespace dcnb {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();  // dcn_forward_plane.cu
+const DeviceInfo *device_info();
+
+namespace {
+
+constexpr int kGStages = 4;
+constexpr int kBM = 128;                 // pixels per tile (the MMA's M)
+constexpr int kBK = 64;                  // channels per K-block (128 bytes: one swizzle row)
+constexpr int kABytes = kBM * kBK * 2;   // 16 KB
+constexpr int kGThreads = 6 * 32;
+
+struct GemmParams {
+    long long P;       // pixels (rows of core and out)
+    int KD, Cout;      // contraction length, output channels
+    int BN;            // output channels per tile (multiple of 16, <= 256)
+    int NT;            // output-channel tiles
+    long long tiles;   // pixel tiles * NT
+    int n_cta;
+    int tmem_cols;     // 2 * BN rounded up to a power of two
+    const void *bias;  // [Cout] or nullptr
+    void *out;
+    unsigned int *err;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kGThreads, 1)
+    proj_gemm_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+                     const GemmParams p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // 1024-byte alignment of the swizzled tiles
+    unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const int stage_bytes = kABytes + p.BN * kBK * 2;
+    unsigned char *ring = smem;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + kGStages * stage_bytes);
+    // full[s], empty[s], acc_full[2], acc_empty[2], drain
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kGStages + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * kGStages;
+    const uint32_t accf0 = empty0 + 8 * kGStages, acce0 = accf0 + 16, drain = acce0 + 16;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KB = p.KD / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kGStages; ++i) {
+            mbar_init(full0 + 8 * i, 1);
+            mbar_init(empty0 + 8 * i, 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(accf0 + 8 * i, 1);
+            mbar_init(acce0 + 8 * i, 4);  // one arrival per epilogue warp
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(p.tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---- producer: A (pixels) and B (weight) K-blocks of every tile of this CTA
+        if (lane == 0) {
+            uint32_t s = 0, pass = 0;
+            long long issued = 0;
+            const uint32_t tx = (uint32_t)stage_bytes;
+            for (long long t = blockIdx.x; t < p.tiles && !*abort_flag; t += p.n_cta) {
+                const int pt = (int)(t / p.NT), nt = (int)(t % p.NT);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (pass >= 1 && !wait_or_abort(empty0 + 8 * s, (pass - 1) & 1, abort_flag)) {
+                        raise_abort(abort_flag, p.err);
+                        break;
+                    }
+                    const uint32_t dst = smem_u32(ring + s * stage_bytes);
+                    mbar_arrive_expect_tx(full0 + 8 * s, tx);
+                    tma_load_2d(dst, &amap, full0 + 8 * s, kb * kBK, pt * kBM);
+                    tma_load_2d(dst + kABytes, &bmap, full0 + 8 * s, kb * kBK, nt * p.BN);
+                    ++issued;
+                    if (++s == kGStages) {
+                        s = 0;
+                        ++pass;
+                    }
+                }
+            }
+            // drain: the last load of every stage has landed before the CTA may exit
+            for (long long j = issued - 1; j >= 0 && j >= issued - kGStages; --j)
+                mbar_wait_bounded(full0 + 8 * (uint32_t)(j % kGStages), (uint32_t)(j / kGStages) & 1, kTcWaitNs);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---- one thread issues the products
+        if (lane == 0) {
+            const int fmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
+            const uint32_t idesc = instr_desc_f16(fmt, p.BN);
+            const uint64_t d0 = smem_desc_sw128(smem_u32(ring));
+            const uint32_t sstep = (uint32_t)stage_bytes >> 4, bofs = (uint32_t)kABytes >> 4;
+            uint32_t s = 0, ph = 0;
+            int local = 0;
+            bool ok = true, issued = false;
+            for (long long t = blockIdx.x; t < p.tiles && ok; t += p.n_cta, ++local) {
+                const int buf = local & 1;
+                // the epilogue has emptied this accumulator (used two tiles ago)
+                if (local >= 2 && !wait_or_abort(acce0 + 8 * buf, ((local >> 1) - 1) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t dcol = tmem + (uint32_t)(buf * p.BN);
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!wait_or_abort(full0 + 8 * s, ph, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = d0 + s * sstep, bd = ad + bofs;
+                    // k-steps of 16 elements = 32 bytes = 2 descriptor units
+                    mma_f16(dcol, ad, bd, idesc, kb != 0);
+                    mma_f16(dcol, ad + 2, bd + 2, idesc, 1u);
+                    mma_f16(dcol, ad + 4, bd + 4, idesc, 1u);
+                    mma_f16(dcol, ad + 6, bd + 6, idesc, 1u);
+                    issued = true;
+                    mma_commit(empty0 + 8 * s);  // stage free once these products are done
+                    if (++s == kGStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(accf0 + 8 * buf);  // accumulator complete
+            }
+            if (!ok) raise_abort(abort_flag, p.err);
+            if (issued) {
+                // every product this thread issued has finished before tensor memory is freed
+                mma_commit(drain);
+                mbar_wait_bounded(drain, 0, kTcWaitNs);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ---- epilogue: warp w reads tensor-memory lanes 32*(w % 4) .. +31 = pixel rows of the tile
+        const int quad = warp & 3;
+        const T *bias = static_cast<const T *>(p.bias);
+        T *out = static_cast<T *>(p.out);
+        int local = 0;
+        for (long long t = blockIdx.x; t < p.tiles; t += p.n_cta, ++local) {
+            const int buf = local & 1;
+            if (!wait_or_abort(accf0 + 8 * buf, (local >> 1) & 1, abort_flag)) {
+                raise_abort(abort_flag, p.err);
+                break;
+            }
+            tc_fence_after();
+            const int pt = (int)(t / p.NT), nt = (int)(t % p.NT);
+            const long long row = (long long)pt * kBM + quad * 32 + lane;
+            for (int c = 0; c < p.BN; c += 16) {
+                float v[16];
+                tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(buf * p.BN + c), v);
+                const int o0 = nt * p.BN + c;
+                if (o0 >= p.Cout) continue;  // warp-uniform
+                if (bias) {  // 16 (or, at the end of an odd Cout, 8) bias values, fp32
+                    float bv[16];
+                    unpack16<T>(ld_nc16(bias + o0), bv);
+                    if (o0 + 16 <= p.Cout) unpack16<T>(ld_nc16(bias + o0 + 8), bv + 8);
+                    else
+#pragma unroll
+                        for (int i = 8; i < 16; ++i) bv[i] = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] += bv[i];
+                }
+                if (row < p.P) {
+                    T *dst = out + row * p.Cout + o0;
+                    if (o0 + 16 <= p.Cout) {
+                        reinterpret_cast<uint4 *>(dst)[0] = pack16<T>(v);
+                        reinterpret_cast<uint4 *>(dst)[1] = pack16<T>(v + 8);
+                    } else {  // Cout is a multiple of 8: one 16-byte half
+                        reinterpret_cast<uint4 *>(dst)[0] = pack16<T>(v);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce0 + 8 * buf);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(p.tmem_cols)
+                     : "memory");
+    }
+}
+
+template <typename T>
+cudaError_t launch_t(const void *core, const void *weight, const void *bias, void *out, long long P, int KD,
+                     int Cout, cudaStream_t stream) {
+    auto enc = encode_fn();
+    const DeviceInfo *dev = device_info();
+    if (!enc || !dev) return cudaErrorNotSupported;
+    GemmParams p;
+    p.P = P;
+    p.KD = KD;
+    p.Cout = Cout;
+    const int c16 = (Cout + 15) & ~15;
+    p.BN = c16 <= 256 ? c16 : 256;
+    p.NT = (Cout + p.BN - 1) / p.BN;
+    p.tiles = ((P + kBM - 1) / kBM) * p.NT;
+    p.n_cta = (int)(p.tiles < dev->sms ? p.tiles : dev->sms);
+    int cols = 32;
+    while (cols < 2 * p.BN) cols <<= 1;
+    p.tmem_cols = cols;
+    p.bias = bias;
+    p.out = out;
+    p.err = dev->err;
+
+    CUtensorMap amap, bmap;
+    const cuuint32_t estr[2] = {1, 1};
+    const cuuint64_t adims[2] = {(cuuint64_t)KD, (cuuint64_t)P};
+    const cuuint64_t astr[1] = {(cuuint64_t)KD * 2};
+    const cuuint32_t abox[2] = {(cuuint32_t)kBK, (cuuint32_t)kBM};
+    const cuuint64_t bdims[2] = {(cuuint64_t)KD, (cuuint64_t)Cout};
+    const cuuint64_t bstr[1] = {(cuuint64_t)KD * 2};
+    const cuuint32_t bbox[2] = {(cuuint32_t)kBK, (cuuint32_t)p.BN};
+    const CUtensorMapDataType dt = std::is_same<T, __half>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (enc(&amap, dt, 2, const_cast<void *>(core), adims, astr, abox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    if (enc(&bmap, dt, 2, const_cast<void *>(weight), bdims, bstr, bbox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    const size_t smem = 1024 + (size_t)kGStages * (kABytes + p.BN * kBK * 2) + (2 * kGStages + 5) * 8 + 16;
+    auto kern = proj_gemm_kernel<T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<p.n_cta, kGThreads, smem, stream>>>(amap, bmap, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_proj_gemm(const void *core, const void *weight, const void *bias, void *out, long long P, int KD,
+                             int Cout, DType dtype, cudaStream_t stream) {
+    if (P <= 0) return cudaSuccess;
+    switch (dtype) {
+        case DType::F16: return launch_t<__half>(core, weight, bias, out, P, KD, Cout, stream);
+        case DType::BF16: return launch_t<__nv_bfloat16>(core, weight, bias, out, P, KD, Cout, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace dcnb

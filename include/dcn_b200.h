@@ -108,9 +108,9 @@ dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offs
                             const void *mask, void *out, dcn_stream_t stream);
 
 /*
- * Forward core followed by its pointwise projection, in one kernel (the
- * DCNv4 module of the YOLOv11 + DCNv4 article, section 3.2, passes the core's
- * output through a 1x1 convolution with bias):
+ * Forward core followed by its pointwise projection (the DCNv4 module of the
+ * YOLOv11 + DCNv4 article, section 3.2, passes the core's output through a
+ * 1x1 convolution with bias):
  *   out[b, ho, wo, o] = bias[o] + sum_j weight[o, j] * core[b, ho, wo, j],
  *   j = g*C + c over the G*C core channels.
  *   weight [Cout, G*C]        storage dtype (a Conv2d weight without its 1x1 extent)
@@ -120,16 +120,30 @@ dcn_status dcn_core_forward(const dcn_params *p, const void *x, const void *offs
  * (pixel, channel) is accumulated in fp32 and rounded once to the storage
  * dtype (what dcn_core_forward would store); the projection runs on the
  * tensor cores with fp32 accumulation, adds the bias in fp32 and rounds the
- * result once.  The core never reaches device memory.
+ * result once.
+ * workspace (optional): a caller-owned device buffer of at least
+ * dcn_core_forward_proj_workspace_bytes(p) bytes (16-byte aligned).  With
+ * it, the call enqueues two kernels: the core (the same kernels as
+ * dcn_core_forward) writes its rounded output [B*Ho*Wo, G*C] into the
+ * workspace, and a tensor-core GEMM projects it; this is the faster route
+ * where the sampling gather dominates (the YOLO P4 shape).  Without it (NULL
+ * or smaller), one fused kernel runs and the core never reaches device
+ * memory.  Both routes compute the same values up to fp32 summation order.
+ * The workspace holds the core output after the call.
  * Supported: fp16 and bf16 (fp32 returns DCN_ERR_UNSUPPORTED), C <= 64 with
  * G*C a multiple of 64 up to 512, kh*kw <= 25, Cout a multiple of 8 in
  * [8, 512], B*H*W and B*Ho*Wo below 2^31; both mask modes.  x, weight and out
  * 16-byte aligned, offset 4-byte, mask and bias 2-byte.  A NaN sampling
  * position makes every output channel of its pixel NaN.
+ * DCN_ERR_SHAPE for a negative workspace_bytes.
  */
 dcn_status dcn_core_forward_proj(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
                                  const void *mask, const void *weight, const void *bias, void *out,
-                                 dcn_stream_t stream);
+                                 void *workspace, int64_t workspace_bytes, dcn_stream_t stream);
+
+/* Workspace bytes for the two-kernel route of dcn_core_forward_proj: the core
+ * output, B*Ho*Wo*G*C*sizeof(dtype).  -1 for invalid params. */
+int64_t dcn_core_forward_proj_workspace_bytes(const dcn_params *p);
 
 /*
  * Modulated deformable convolution with a dense weight per kernel point (the
@@ -267,10 +281,37 @@ int32_t dcn_take_device_error(void);
  * before.  DCN_ERR_SHAPE for a limit outside the range. */
 dcn_status dcn_selftest_bounded_wait(int32_t limit_us, dcn_stream_t stream);
 
+/*
+ * On-chip rate probes: measurement support for the roofline of the sampling
+ * kernels (the pages have no counterpart).  Runs probe number `probe` on one
+ * CTA of 512 threads per SM, `reps` (1 .. 2^24) repetitions of its loop, on
+ * `stream`:
+ *    0  16-byte shared loads (bytes)
+ *    1  chunk: two 16-byte shared loads of fp32 + 4 paired FMAs (chunks of 8 channels)
+ *    2  fp32 FMAs                          3  paired fp32 FMAs (fma counted)
+ *    4  chunk: 16-byte shared load of fp16 + 8 conversions + 8 FMAs (chunks)
+ *    5  chunk: load + 8 fp16 conversions + 4 paired FMAs (chunks)
+ *    6  chunk: load + bf16 widening by shift and mask + 4 paired FMAs (chunks)
+ *    7  chunk: load + 8 fma.rn.f32.f16 with fp16 operands (chunks)
+ *    8  16-byte global loads hitting L1 (bytes)
+ *    9  gather, 4 lanes per 64-byte item (samples)
+ *   10  gather, 8 lanes per item, paired FMAs (samples)
+ *   11  gather, 8 lanes per item, FMAs (samples)
+ *   12  integer lop3 (ops)
+ * dev_buf is a caller-owned device buffer of at least 36,864 bytes, 256-byte
+ * aligned: on completion its first two 64-bit words hold the sum over the
+ * CTAs of their SM-clock cycles and the number of CTAs (the rest is scratch
+ * of the probe).  *units_per_cta receives the work of one CTA in *unit, so
+ * units per SM per clock = units_per_cta * word[1] / word[0].
+ * DCN_ERR_SHAPE for an unknown probe, reps out of range or a small buffer.
+ */
+dcn_status dcn_probe_rate(int32_t probe, int32_t reps, void *dev_buf, int64_t dev_buf_bytes,
+                          double *units_per_cta, const char **unit, dcn_stream_t stream);
+
 /* ABI version of this header (bumped on any incompatible change). */
 int32_t dcn_abi_version(void);
 
-#define DCN_ABI_VERSION 1
+#define DCN_ABI_VERSION 2
 
 #ifdef __cplusplus
 }

@@ -152,19 +152,24 @@ def test_proj_checks(lib):
     refused on the host (fake, never-dereferenced pointers)."""
     p = params(G=16, C=32)  # fp16, G*C = 512
     f = lib.dcn_core_forward_proj
-    assert f(ctypes.byref(p), 512, 16, 16, 16, 0, None, 16, None) == B.DCN_ERR_NULL          # no weight
-    assert f(ctypes.byref(p), 512, 16, 16, 16, 8, None, 16, None) == B.DCN_ERR_ALIGN         # weight 8-byte
-    assert f(ctypes.byref(p), 512, 16, 16, 16, 16, 3, 16, None) == B.DCN_ERR_ALIGN           # odd bias address
-    assert f(ctypes.byref(p), 100, 16, 16, 16, 16, None, 16, None) == B.DCN_ERR_UNSUPPORTED  # Cout % 8
-    assert f(ctypes.byref(p), 520, 16, 16, 16, 16, None, 16, None) == B.DCN_ERR_UNSUPPORTED  # Cout > 512
+    assert f(ctypes.byref(p), 512, 16, 16, 16, 0, None, 16, None, 0, None) == B.DCN_ERR_NULL          # no weight
+    assert f(ctypes.byref(p), 512, 16, 16, 16, 8, None, 16, None, 0, None) == B.DCN_ERR_ALIGN         # weight 8-byte
+    assert f(ctypes.byref(p), 512, 16, 16, 16, 16, 3, 16, None, 0, None) == B.DCN_ERR_ALIGN           # odd bias
+    assert f(ctypes.byref(p), 100, 16, 16, 16, 16, None, 16, None, 0, None) == B.DCN_ERR_UNSUPPORTED  # Cout % 8
+    assert f(ctypes.byref(p), 520, 16, 16, 16, 16, None, 16, None, 0, None) == B.DCN_ERR_UNSUPPORTED  # Cout > 512
+    assert f(ctypes.byref(p), 512, 16, 16, 16, 16, None, 16, None, -1, None) == B.DCN_ERR_SHAPE       # ws bytes < 0
+    need = lib.dcn_core_forward_proj_workspace_bytes(ctypes.byref(p))
+    assert need == 2 * 40 * 40 * 512 * 2
+    assert f(ctypes.byref(p), 512, 16, 16, 16, 16, None, 16, 8, need, None) == B.DCN_ERR_ALIGN       # ws 8-byte
     for bad in (params(G=16, C=32, dtype=0),     # fp32
                 params(G=3, C=32),               # G*C = 96
                 params(G=32, C=32),              # G*C = 1024
                 params(G=1, C=128),              # C > 64
                 params(G=16, C=32, kh=7, kw=7, pad_h=3, pad_w=3)):  # 49 points
-        assert f(ctypes.byref(bad), 64, 16, 16, 16, 16, None, 16, None) == B.DCN_ERR_UNSUPPORTED
+        assert f(ctypes.byref(bad), 64, 16, 16, 16, 16, None, 16, None, 0, None) == B.DCN_ERR_UNSUPPORTED
     empty = params(B=0, G=16, C=32)
-    assert f(ctypes.byref(empty), 64, None, None, None, None, None, None, None) == B.DCN_OK
+    assert f(ctypes.byref(empty), 64, None, None, None, None, None, None, None, 0, None) == B.DCN_OK
+    assert lib.dcn_core_forward_proj_workspace_bytes(ctypes.byref(params(H=0))) == -1
 
 
 def test_selftest_limit_checked_on_host(lib):
