@@ -28,7 +28,7 @@ EXPORTS = ("dcn_core_output_hw", "dcn_core_forward", "dcn_core_backward", "defor
            "deform_agg_backward", "dcn_status_string", "dcn_last_error_detail", "dcn_abi_version",
            "dcn_take_device_error", "deform_roi_pool_forward", "dcn_core_forward_proj",
            "dcn_selftest_bounded_wait", "dcn_deform_conv_forward", "dcn_probe_rate",
-           "dcn_core_forward_proj_workspace_bytes")
+           "dcn_core_forward_proj_workspace_bytes", "dcn_core_forward_proj_noalloc")
 ABI_VERSION = 2
 
 
@@ -84,6 +84,8 @@ def _declare(lib):
     lib.dcn_core_forward_proj.restype = st
     lib.dcn_core_forward_proj_workspace_bytes.argtypes = [P]
     lib.dcn_core_forward_proj_workspace_bytes.restype = ctypes.c_int64
+    lib.dcn_core_forward_proj_noalloc.argtypes = [P, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp]
+    lib.dcn_core_forward_proj_noalloc.restype = st
     lib.dcn_deform_conv_forward.argtypes = [P, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp]
     lib.dcn_deform_conv_forward.restype = st
     lib.dcn_selftest_bounded_wait.argtypes = [ctypes.c_int32, vp]

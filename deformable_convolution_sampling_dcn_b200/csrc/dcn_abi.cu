@@ -7,6 +7,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "dcn_b200.h"
 #include "dcn_launch.h"
 
@@ -229,6 +231,66 @@ dcn_status dcn_core_forward_proj(const dcn_params *p, int32_t Cout, const void *
     if (workspace_bytes < 0) return fail(DCN_ERR_SHAPE, "workspace_bytes is negative");
     return proj_call(p, Cout, x, offset, mask, weight, bias, out, workspace, workspace_bytes, stream, false,
                      "dcn_core_forward_proj launch");
+}
+
+}  // extern "C"
+
+namespace {
+
+// Scratch of dcn_core_forward_proj_noalloc: a fixed array in device memory,
+// one per GPU that loads the library, kept until the process exits.  Host code
+// may not pass the symbol itself to a kernel (on the host it names a shadow
+// variable, not device memory): noalloc_scratch() looks its device address up
+// once per device, with that device current.
+constexpr size_t kNoAllocScratchBytes = (size_t)DCN_NOALLOC_SCRATCH_BYTES;
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void *noalloc_scratch(cudaError_t *err) {
+    constexpr int kMaxDev = 64;
+    static void *addr[kMaxDev];
+    static cudaError_t status[kMaxDev];
+    static std::once_flag once[kMaxDev];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+        *err = e != cudaSuccess ? e : cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    std::call_once(once[dev], [dev] {
+        void *p = nullptr;
+        status[dev] = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        addr[dev] = status[dev] == cudaSuccess ? p : nullptr;
+    });
+    *err = status[dev];
+    return addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+dcn_status dcn_core_forward_proj_noalloc(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
+                                         const void *mask, const void *weight, const void *bias, void *out,
+                                         dcn_stream_t stream) {
+    const long long need = core_out_bytes(p);
+    if (need < 0) {
+        int Ho = 0, Wo = 0;
+        return check_core(p, &Ho, &Wo);  // the same status and detail as the other calls
+    }
+    if ((size_t)need > kNoAllocScratchBytes)
+        return fail(DCN_ERR_UNSUPPORTED,
+                    "dcn_core_forward_proj_noalloc: the core output needs %lld bytes, more than its fixed "
+                    "%zu-byte scratch; use dcn_core_forward_proj with a workspace",
+                    need, kNoAllocScratchBytes);
+    if (p->B == 0) return proj_call(p, Cout, x, offset, mask, weight, bias, out, nullptr, 0, stream, false,
+                                    "dcn_core_forward_proj_noalloc");
+    cudaError_t e = cudaSuccess;
+    void *scratch = noalloc_scratch(&e);
+    if (!scratch) return cuda_status(e == cudaSuccess ? cudaErrorInvalidSymbol : e,
+                                     "dcn_core_forward_proj_noalloc scratch address");
+    // the workspace route of dcn_core_forward_proj with the fixed array as workspace
+    return proj_call(p, Cout, x, offset, mask, weight, bias, out, scratch, (int64_t)kNoAllocScratchBytes, stream,
+                     false, "dcn_core_forward_proj_noalloc launch");
 }
 
 int64_t dcn_core_forward_proj_workspace_bytes(const dcn_params *p) {

@@ -146,6 +146,34 @@ dcn_status dcn_core_forward_proj(const dcn_params *p, int32_t Cout, const void *
 int64_t dcn_core_forward_proj_workspace_bytes(const dcn_params *p);
 
 /*
+ * dcn_core_forward_proj for callers that cannot allocate device memory (this
+ * entry point is the library's own addition; the pages have no counterpart).
+ * Some callers have no way to obtain a workspace: a plugin hosted by a
+ * framework or serving runtime whose allocator owns all of the GPU's memory
+ * gets no handle to it, and a latency-critical loop cannot afford the
+ * device-wide synchronisation that cudaMalloc implies.  This call allocates
+ * nothing: it runs the workspace route of dcn_core_forward_proj (core kernel,
+ * then the tensor-core GEMM) with a fixed scratch array of
+ * DCN_NOALLOC_SCRATCH_BYTES (16 MiB) that the library holds in the memory of
+ * every GPU that loads it, until the process exits.  The caller still owns
+ * x, offset, mask, weight, bias and out, with the rules of
+ * dcn_core_forward_proj.
+ * Limit: the core output B*Ho*Wo*G*C*sizeof(dtype) must fit the array (the
+ * DCNv4 P4 batch of 8 needs 13,107,200 bytes); a larger problem returns
+ * DCN_ERR_UNSUPPORTED with a detail naming both sizes, before any launch.
+ * Every call on a device shares the one array and leaves the core output of
+ * its problem in it (every byte it reads is written by the same call first):
+ * calls whose kernels overlap on the GPU, e.g. on two streams, race on it and
+ * give wrong results; order them.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress, once per device, with that
+ * device current); make that first call before any stream capture.
+ */
+#define DCN_NOALLOC_SCRATCH_BYTES (16 * 1024 * 1024)
+dcn_status dcn_core_forward_proj_noalloc(const dcn_params *p, int32_t Cout, const void *x, const void *offset,
+                                         const void *mask, const void *weight, const void *bias, void *out,
+                                         dcn_stream_t stream);
+
+/*
  * Modulated deformable convolution with a dense weight per kernel point (the
  * DCNv2 page "DCNv2实战：在YOLOv5中替换普通卷积...", section 1:
  * y(p0) = sum_n w(pn) * x(p0 + pn + dpn) * dm_n; with unit masks it is the DCNv1
