@@ -37,10 +37,26 @@ constexpr int kBK = 64;                  // channels per K-block (128 bytes: one
 constexpr int kABytes = kBM * kBK * 2;   // 16 KB
 constexpr int kGThreads = 6 * 32;
 
+// 32 consecutive fp32 accumulator columns of this warp's 32 tensor-memory lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 struct GemmParams {
     long long P;       // pixels (rows of core and out)
     int KD, Cout;      // contraction length, output channels
-    int BN;            // output channels per tile (multiple of 16, <= 256)
+    int BN;            // output channels per tile (multiple of 32, <= 256)
     int NT;            // output-channel tiles
     long long tiles;   // pixel tiles * NT
     int n_cta;
@@ -63,6 +79,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     // full[s], empty[s], acc_full[2], acc_empty[2], drain
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kGStages + 5);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float *bias_s = reinterpret_cast<float *>(tmem_slot + 6);  // [NT * BN] fp32, zero past Cout (16-byte aligned)
     const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * kGStages;
     const uint32_t accf0 = empty0 + 8 * kGStages, acce0 = accf0 + 16, drain = acce0 + 16;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -175,6 +192,10 @@ __global__ void __launch_bounds__(kGThreads, 1)
         const int quad = warp & 3;
         const T *bias = static_cast<const T *>(p.bias);
         T *out = static_cast<T *>(p.out);
+        // the bias, once per CTA, in fp32 (zero past Cout or without bias)
+        for (int i = threadIdx.x - 64; i < p.NT * p.BN; i += 128)
+            bias_s[i] = (bias && i < p.Cout) ? to_f32(bias[i]) : 0.0f;
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
         int local = 0;
         for (long long t = blockIdx.x; t < p.tiles; t += p.n_cta, ++local) {
             const int buf = local & 1;
@@ -185,29 +206,26 @@ __global__ void __launch_bounds__(kGThreads, 1)
             tc_fence_after();
             const int pt = (int)(t / p.NT), nt = (int)(t % p.NT);
             const long long row = (long long)pt * kBM + quad * 32 + lane;
-            for (int c = 0; c < p.BN; c += 16) {
-                float v[16];
-                tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(buf * p.BN + c), v);
+            for (int c = 0; c < p.BN; c += 32) {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(buf * p.BN + c), v);
                 const int o0 = nt * p.BN + c;
                 if (o0 >= p.Cout) continue;  // warp-uniform
-                if (bias) {  // 16 (or, at the end of an odd Cout, 8) bias values, fp32
-                    float bv[16];
-                    unpack16<T>(ld_nc16(bias + o0), bv);
-                    if (o0 + 16 <= p.Cout) unpack16<T>(ld_nc16(bias + o0 + 8), bv + 8);
-                    else
+                const float4 *bb = reinterpret_cast<const float4 *>(bias_s + o0);
 #pragma unroll
-                        for (int i = 8; i < 16; ++i) bv[i] = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] += bv[i];
+                for (int i = 0; i < 8; ++i) {
+                    const float4 b4 = bb[i];
+                    v[4 * i] += b4.x;
+                    v[4 * i + 1] += b4.y;
+                    v[4 * i + 2] += b4.z;
+                    v[4 * i + 3] += b4.w;
                 }
                 if (row < p.P) {
                     T *dst = out + row * p.Cout + o0;
-                    if (o0 + 16 <= p.Cout) {
-                        reinterpret_cast<uint4 *>(dst)[0] = pack16<T>(v);
-                        reinterpret_cast<uint4 *>(dst)[1] = pack16<T>(v + 8);
-                    } else {  // Cout is a multiple of 8: one 16-byte half
-                        reinterpret_cast<uint4 *>(dst)[0] = pack16<T>(v);
-                    }
+                    const int n16 = (p.Cout - o0) >= 32 ? 4 : (p.Cout - o0) / 8;  // Cout is a multiple of 8
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if (i < n16) reinterpret_cast<uint4 *>(dst)[i] = pack16<T>(v + 8 * i);
                 }
             }
             tc_fence_before();
@@ -234,8 +252,9 @@ cudaError_t launch_t(const void *core, const void *weight, const void *bias, voi
     p.P = P;
     p.KD = KD;
     p.Cout = Cout;
-    const int c16 = (Cout + 15) & ~15;
-    p.BN = c16 <= 256 ? c16 : 256;
+    // a multiple of 32, so the epilogue's 32-column loads stay inside the tile
+    const int c32 = (Cout + 31) & ~31;
+    p.BN = c32 <= 256 ? c32 : 256;
     p.NT = (Cout + p.BN - 1) / p.BN;
     p.tiles = ((P + kBM - 1) / kBM) * p.NT;
     p.n_cta = (int)(p.tiles < dev->sms ? p.tiles : dev->sms);
@@ -264,7 +283,8 @@ cudaError_t launch_t(const void *core, const void *weight, const void *bias, voi
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const size_t smem = 1024 + (size_t)kGStages * (kABytes + p.BN * kBK * 2) + (2 * kGStages + 5) * 8 + 16;
+    const size_t smem = 1024 + (size_t)kGStages * (kABytes + p.BN * kBK * 2) + (2 * kGStages + 5) * 8 + 32 +
+                        (size_t)p.NT * p.BN * 4;
     auto kern = proj_gemm_kernel<T>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
