@@ -21,8 +21,15 @@ def test_traffic_record_matches_kernel_sources():
 
 
 def test_profiles_give_their_commands():
+    """Every summary gives the command that made it, in a fenced block, running
+    committed files only; every ncu command in it leaves the GPU clocks alone."""
     d = os.path.join(ROOT, "profiles")
     for name in os.listdir(d):
         if name.endswith(".md"):
             text = open(os.path.join(d, name), encoding="utf-8").read()
-            assert "ncu " in text and "--clock-control none" in text, name
+            blocks = text.split("```")[1::2]
+            assert blocks and any(("bench.py" in b) or ("python -c" in b) for b in blocks), name
+            for b in blocks:
+                if "ncu " in b:
+                    assert "--clock-control none" in b, name
+                assert "_work" not in b, name
