@@ -237,7 +237,7 @@ def run_ours(args, world, rank, local):
             tr = json.load(f)
         ent = tr.get("dcnv4_p4_forward")
         if ent and ent.get("kernel_hash") == kernel_hash():
-            traffic = ent["dram_bytes_per_launch"]
+            traffic = ent["bytes_per_launch"]  # DRAM reads + the launch's L2 writes (its output)
             insts = ent.get("warp_instructions_per_launch")
             if insts and clocks.get("sm_mhz"):
                 # the ceiling that binds this gather: one warp instruction per

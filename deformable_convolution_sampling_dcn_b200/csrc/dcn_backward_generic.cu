@@ -1,13 +1,7 @@
 // Generic backward core: any shape the ABI accepts, global atomic scatter.
 //
-// One LPI-lane sub-warp per (pixel, group) item, 16 bytes of channels per
-// lane.  Items are taken in plane-major order ((b, g) planes, pixels inside
-// a plane row by row) and the grid is persistent: CTA c owns the contiguous
-// item range [T*c/NC, T*(c+1)/NC) and its warps step through it together, so
-// the taps an SM issues at any moment fall on a few neighbouring rows of one
-// group's input plane and mostly hit L1 (with the pixel-major, grid-stride
-// order each warp sampled a different group and most corner reads went to
-// L2, where they compete with the input-gradient reductions).  Per tap each lane forms
+// Same item mapping as the generic forward (one LPI-lane sub-warp per
+// (pixel, group), 16 bytes of channels per lane).  Per tap each lane forms
 // the dot products d_c = <grad_out, x(corner c)> over its channels for the
 // four corners; the sample value and its two position derivatives are
 // linear combinations of the d_c:
@@ -24,10 +18,8 @@
 namespace dcnb {
 namespace {
 
-constexpr int kBwdThreads = 256;
-
 template <typename T, int LPI, bool SOFTMAX>
-__global__ void __launch_bounds__(kBwdThreads) core_backward_generic(CoreArgs a, ItemDecode dd) {
+__global__ void __launch_bounds__(256) core_backward_generic(CoreArgs a, ItemDecode dd) {
     constexpr int V = Storage<T>::kVec;
     constexpr int IPW = 32 / LPI;
     const int lane = threadIdx.x & 31;
@@ -36,10 +28,7 @@ __global__ void __launch_bounds__(kBwdThreads) core_backward_generic(CoreArgs a,
     const int K = a.kh * a.kw;
     const int GC = a.G * a.C;
     const long long n_items = (long long)a.B * a.Ho * a.Wo * a.G;
-    const long long hw = (long long)a.Ho * a.Wo;
-    // this CTA's contiguous item range; its warps take IPW items each, in step
-    const long long r0 = n_items * blockIdx.x / gridDim.x, r1 = n_items * (blockIdx.x + 1) / gridDim.x;
-    const long long cta_step = (long long)(blockDim.x >> 5) * IPW;
+    const long long warps_total = (long long)gridDim.x * (blockDim.x >> 5);
     const T *__restrict__ x = static_cast<const T *>(a.x);
     const T *__restrict__ off = static_cast<const T *>(a.offset);
     const T *__restrict__ msk = static_cast<const T *>(a.mask);
@@ -51,30 +40,29 @@ __global__ void __launch_bounds__(kBwdThreads) core_backward_generic(CoreArgs a,
 
     // Warp-uniform loop: every lane runs the same iterations so that the
     // sub-warp shuffles always see all 32 lanes.
-    for (long long base = r0 + (long long)(threadIdx.x >> 5) * IPW; base < r1; base += cta_step) {
-        const long long item = base + slot;  // plane-major: ((b*G + g)*Ho + ho)*Wo + wo
-        const bool active = item < r1;
-        const long long pm = active ? item : r0;
+    for (long long base = ((long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * IPW;
+         base < n_items; base += warps_total * IPW) {
+        const long long item = base + slot;
+        const bool active = item < n_items;
+        const long long it = active ? item : 0;
         int g, wo, ho, b;
         if (n_items < (1LL << 31)) {  // 32-bit decode by multiply-high (the common case)
             unsigned r;
-            unsigned t = fdiv((unsigned)pm, dd.wo, r);
-            wo = (int)r;
-            t = fdiv(t, dd.ho, r);
-            ho = (int)r;
-            b = (int)fdiv(t, dd.g, r);
+            unsigned t = fdiv((unsigned)it, dd.g, r);
             g = (int)r;
+            t = fdiv(t, dd.wo, r);
+            wo = (int)r;
+            b = (int)fdiv(t, dd.ho, r);
+            ho = (int)r;
         } else {
-            long long t = pm;
+            long long t = it;
+            g = (int)(t % a.G);
+            t /= a.G;
             wo = (int)(t % a.Wo);
             t /= a.Wo;
             ho = (int)(t % a.Ho);
-            t /= a.Ho;
-            g = (int)(t % a.G);
-            b = (int)(t / a.G);
+            b = (int)(t / a.Ho);
         }
-        // index of the item in the [B, Ho, Wo, G] layout of offset, mask and their gradients
-        const long long it = ((long long)b * hw + (long long)ho * a.Wo + wo) * a.G + g;
         const T *o_item = off + it * K * 2;
         const T *m_item = msk + it * K;
 
@@ -169,17 +157,10 @@ __global__ void __launch_bounds__(kBwdThreads) core_backward_generic(CoreArgs a,
 template <typename T, int LPI>
 cudaError_t launch_lpi(const CoreArgs &a, cudaStream_t stream) {
     const long long n_items = (long long)a.B * a.Ho * a.Wo * a.G;
-    const int threads = kBwdThreads;
+    const int threads = 256;
     const long long items_per_block = (threads / 32) * (32 / LPI);
-    // persistent: as many CTAs as fit on the SMs at once, each with a long contiguous item range
-    int sms = 148, per_sm = 1, dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    auto kern = a.softmax ? core_backward_generic<T, LPI, true> : core_backward_generic<T, LPI, false>;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess || per_sm < 1)
-        per_sm = 1;
-    long long blocks = (long long)sms * per_sm;
-    const long long need = (n_items + items_per_block - 1) / items_per_block;
-    if (blocks > need) blocks = need;
+    long long blocks = (n_items + items_per_block - 1) / items_per_block;
+    if (blocks > 148LL * 64) blocks = 148LL * 64;
     const ItemDecode dd = make_item_decode(a.G, a.Wo, a.Ho);
     if (a.softmax)
         core_backward_generic<T, LPI, true><<<(unsigned)blocks, threads, 0, stream>>>(a, dd);
