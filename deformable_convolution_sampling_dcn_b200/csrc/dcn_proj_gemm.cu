@@ -6,10 +6,13 @@
 // core [P, KD] and weight [Cout, KD] are both K-major (row-major with the
 // contraction index fastest), fp16 or bf16; out [P, Cout] in the same type.
 //
-// Persistent, warp-specialised: warp 0 streams (pixel tile, weight tile)
-// K-blocks of 64 channels by TMA (128-byte swizzle) through a 4-stage ring,
-// one thread of warp 1 issues tcgen05.mma (M = 128 pixels, N = up to 256
-// output channels, K = 16) into one of two tensor-memory accumulators, and
+// Persistent, warp-specialised: every CTA works on one tile of up to 128
+// output channels, whose weight rows (all K-blocks, at most 128 KB) warp 0
+// loads once into shared memory by TMA; it then streams the CTA's pixel
+// tiles, K-block by K-block (64 channels, 128-byte swizzle), through a
+// 4-stage ring.  One thread of warp 1 issues tcgen05.mma (M = 128 pixels,
+// N = up to 128 output channels, K = 16) into one of two tensor-memory
+// accumulators, and
 // warps 2..5 (one per 32-lane quarter of tensor memory) read the finished
 // accumulator back with tcgen05.ld, add the bias in fp32, round once to the
 // storage type and store, while the products of the next tile already run
@@ -35,6 +38,8 @@ constexpr int kGStages = 4;
 constexpr int kBM = 128;                 // pixels per tile (the MMA's M)
 constexpr int kBK = 64;                  // channels per K-block (128 bytes: one swizzle row)
 constexpr int kABytes = kBM * kBK * 2;   // 16 KB
+constexpr int kBNMax = 128;              // output channels per tile (resident weight rows)
+constexpr int kMaxKB = 8;                // K-blocks of the contraction (G*C <= 512)
 constexpr int kGThreads = 6 * 32;
 
 // 32 consecutive fp32 accumulator columns of this warp's 32 tensor-memory lanes.
@@ -56,10 +61,10 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
 struct GemmParams {
     long long P;       // pixels (rows of core and out)
     int KD, Cout;      // contraction length, output channels
-    int BN;            // output channels per tile (multiple of 32, <= 256)
+    int BN;            // output channels per tile (multiple of 32, <= 128)
     int NT;            // output-channel tiles
-    long long tiles;   // pixel tiles * NT
-    int n_cta;
+    long long PT;      // pixel tiles
+    int n_cta;         // a multiple of NT: CTA c works on output-channel tile c % NT
     int tmem_cols;     // 2 * BN rounded up to a power of two
     const void *bias;  // [Cout] or nullptr
     void *out;
@@ -73,17 +78,21 @@ __global__ void __launch_bounds__(kGThreads, 1)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment of the swizzled tiles
     unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    const int stage_bytes = kABytes + p.BN * kBK * 2;
-    unsigned char *ring = smem;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + kGStages * stage_bytes);
-    // full[s], empty[s], acc_full[2], acc_empty[2], drain
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kGStages + 5);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float *bias_s = reinterpret_cast<float *>(tmem_slot + 6);  // [NT * BN] fp32, zero past Cout (16-byte aligned)
-    const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * kGStages;
-    const uint32_t accf0 = empty0 + 8 * kGStages, acce0 = accf0 + 16, drain = acce0 + 16;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int KB = p.KD / kBK;
+    const int wblk = p.BN * kBK * 2;  // one resident weight K-block
+    unsigned char *wres = smem;       // [KB][BN rows x 128 bytes], swizzled
+    unsigned char *ring = smem + KB * wblk;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + kGStages * kABytes);
+    // full[s], empty[s], acc_full[2], acc_empty[2], drain, weights[kMaxKB] (one per resident K-block)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kGStages + 5 + kMaxKB);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    // [NT * BN] fp32 bias, zero past Cout, at the next 16-byte boundary after the slot and the flag
+    float *bias_s = reinterpret_cast<float *>((reinterpret_cast<uintptr_t>(tmem_slot + 2) + 15) & ~(uintptr_t)15);
+    const uint32_t full0 = smem_u32(bars), empty0 = full0 + 8 * kGStages;
+    const uint32_t accf0 = empty0 + 8 * kGStages, acce0 = accf0 + 16, drain = acce0 + 16, wfull = drain + 8;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nt = blockIdx.x % p.NT;  // this CTA's output-channel tile
+    const long long pt0 = blockIdx.x / p.NT, pstep = p.n_cta / p.NT;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kGStages; ++i) {
@@ -95,6 +104,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
             mbar_init(acce0 + 8 * i, 4);  // one arrival per epilogue warp
         }
         mbar_init(drain, 1);
+        for (int i = 0; i < kMaxKB; ++i) mbar_init(wfull + 8 * i, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -110,22 +120,32 @@ __global__ void __launch_bounds__(kGThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ---- producer: A (pixels) and B (weight) K-blocks of every tile of this CTA
+        // ---- producer: this CTA's weight rows once, then the pixel K-blocks of its tiles
         if (lane == 0) {
             uint32_t s = 0, pass = 0;
             long long issued = 0;
-            const uint32_t tx = (uint32_t)stage_bytes;
-            for (long long t = blockIdx.x; t < p.tiles && !*abort_flag; t += p.n_cta) {
-                const int pt = (int)(t / p.NT), nt = (int)(t % p.NT);
+            int wissued = 0;  // weight K-blocks issued
+            bool first = true;
+            for (long long pt = pt0; pt < p.PT && !*abort_flag; pt += pstep, first = false) {
                 for (int kb = 0; kb < KB; ++kb) {
+                    // first tile: weight K-block kb just ahead of pixel K-block kb while the ring
+                    // fills, then every remaining weight K-block at once
+                    if (first && kb < kGStages) {
+                        mbar_arrive_expect_tx(wfull + 8 * kb, (uint32_t)wblk);
+                        tma_load_2d(smem_u32(wres + kb * wblk), &bmap, wfull + 8 * kb, kb * kBK, nt * p.BN);
+                        ++wissued;
+                    }
+                    if (first && kb == kGStages)
+                        for (int j = kGStages; j < KB; ++j, ++wissued) {
+                            mbar_arrive_expect_tx(wfull + 8 * j, (uint32_t)wblk);
+                            tma_load_2d(smem_u32(wres + j * wblk), &bmap, wfull + 8 * j, j * kBK, nt * p.BN);
+                        }
                     if (pass >= 1 && !wait_or_abort(empty0 + 8 * s, (pass - 1) & 1, abort_flag)) {
                         raise_abort(abort_flag, p.err);
                         break;
                     }
-                    const uint32_t dst = smem_u32(ring + s * stage_bytes);
-                    mbar_arrive_expect_tx(full0 + 8 * s, tx);
-                    tma_load_2d(dst, &amap, full0 + 8 * s, kb * kBK, pt * kBM);
-                    tma_load_2d(dst + kABytes, &bmap, full0 + 8 * s, kb * kBK, nt * p.BN);
+                    mbar_arrive_expect_tx(full0 + 8 * s, (uint32_t)kABytes);
+                    tma_load_2d(smem_u32(ring + s * kABytes), &amap, full0 + 8 * s, kb * kBK, (int)pt * kBM);
                     ++issued;
                     if (++s == kGStages) {
                         s = 0;
@@ -133,7 +153,8 @@ __global__ void __launch_bounds__(kGThreads, 1)
                     }
                 }
             }
-            // drain: the last load of every stage has landed before the CTA may exit
+            // drain: the weights and the last load of every stage have landed before the CTA may exit
+            for (int kb = 0; kb < wissued; ++kb) mbar_wait_bounded(wfull + 8 * kb, 0, kTcWaitNs);
             for (long long j = issued - 1; j >= 0 && j >= issued - kGStages; --j)
                 mbar_wait_bounded(full0 + 8 * (uint32_t)(j % kGStages), (uint32_t)(j / kGStages) & 1, kTcWaitNs);
         }
@@ -143,12 +164,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (lane == 0) {
             const int fmt = std::is_same<T, __nv_bfloat16>::value ? 1 : 0;
             const uint32_t idesc = instr_desc_f16(fmt, p.BN);
-            const uint64_t d0 = smem_desc_sw128(smem_u32(ring));
-            const uint32_t sstep = (uint32_t)stage_bytes >> 4, bofs = (uint32_t)kABytes >> 4;
+            const uint64_t a0 = smem_desc_sw128(smem_u32(ring)), b0 = smem_desc_sw128(smem_u32(wres));
+            const uint32_t sstep = (uint32_t)kABytes >> 4, wstep = (uint32_t)wblk >> 4;
             uint32_t s = 0, ph = 0;
             int local = 0;
             bool ok = true, issued = false;
-            for (long long t = blockIdx.x; t < p.tiles && ok; t += p.n_cta, ++local) {
+            for (long long pt = pt0; pt < p.PT && ok; pt += pstep, ++local) {
                 const int buf = local & 1;
                 // the epilogue has emptied this accumulator (used two tiles ago)
                 if (local >= 2 && !wait_or_abort(acce0 + 8 * buf, ((local >> 1) - 1) & 1, abort_flag)) {
@@ -158,12 +179,13 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 tc_fence_after();
                 const uint32_t dcol = tmem + (uint32_t)(buf * p.BN);
                 for (int kb = 0; kb < KB; ++kb) {
-                    if (!wait_or_abort(full0 + 8 * s, ph, abort_flag)) {
+                    if ((local == 0 && !wait_or_abort(wfull + 8 * kb, 0, abort_flag)) ||
+                        !wait_or_abort(full0 + 8 * s, ph, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint64_t ad = d0 + s * sstep, bd = ad + bofs;
+                    const uint64_t ad = a0 + s * sstep, bd = b0 + kb * wstep;
                     // k-steps of 16 elements = 32 bytes = 2 descriptor units
                     mma_f16(dcol, ad, bd, idesc, kb != 0);
                     mma_f16(dcol, ad + 2, bd + 2, idesc, 1u);
@@ -197,15 +219,14 @@ __global__ void __launch_bounds__(kGThreads, 1)
             bias_s[i] = (bias && i < p.Cout) ? to_f32(bias[i]) : 0.0f;
         asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
         int local = 0;
-        for (long long t = blockIdx.x; t < p.tiles; t += p.n_cta, ++local) {
+        for (long long pt = pt0; pt < p.PT; pt += pstep, ++local) {
             const int buf = local & 1;
             if (!wait_or_abort(accf0 + 8 * buf, (local >> 1) & 1, abort_flag)) {
                 raise_abort(abort_flag, p.err);
                 break;
             }
             tc_fence_after();
-            const int pt = (int)(t / p.NT), nt = (int)(t % p.NT);
-            const long long row = (long long)pt * kBM + quad * 32 + lane;
+            const long long row = pt * kBM + quad * 32 + lane;
             for (int c = 0; c < p.BN; c += 32) {
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(buf * p.BN + c), v);
@@ -254,10 +275,13 @@ cudaError_t launch_t(const void *core, const void *weight, const void *bias, voi
     p.Cout = Cout;
     // a multiple of 32, so the epilogue's 32-column loads stay inside the tile
     const int c32 = (Cout + 31) & ~31;
-    p.BN = c32 <= 256 ? c32 : 256;
+    p.BN = c32 <= kBNMax ? c32 : kBNMax;
     p.NT = (Cout + p.BN - 1) / p.BN;
-    p.tiles = ((P + kBM - 1) / kBM) * p.NT;
-    p.n_cta = (int)(p.tiles < dev->sms ? p.tiles : dev->sms);
+    p.PT = (P + kBM - 1) / kBM;
+    long long per_nt = dev->sms / p.NT;  // CTAs per output-channel tile
+    if (per_nt > p.PT) per_nt = p.PT;
+    if (per_nt < 1) per_nt = 1;
+    p.n_cta = (int)(per_nt * p.NT);
     int cols = 32;
     while (cols < 2 * p.BN) cols <<= 1;
     p.tmem_cols = cols;
@@ -283,8 +307,8 @@ cudaError_t launch_t(const void *core, const void *weight, const void *bias, voi
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const size_t smem = 1024 + (size_t)kGStages * (kABytes + p.BN * kBK * 2) + (2 * kGStages + 5) * 8 + 32 +
-                        (size_t)p.NT * p.BN * 4;
+    const size_t smem = 1024 + (size_t)(KD / kBK) * p.BN * kBK * 2 + (size_t)kGStages * kABytes +
+                        (2 * kGStages + 5 + kMaxKB) * 8 + 32 + (size_t)p.NT * p.BN * 4;
     auto kern = proj_gemm_kernel<T>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
