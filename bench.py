@@ -699,7 +699,8 @@ def run_ceilings(reps_scale: float) -> None:
     # repetitions giving a few milliseconds per probe
     reps = {"lds128": 20000, "chunk_f32_ffma2": 80000, "ffma": 20000, "ffma2": 20000, "chunk_f16_ffma": 80000,
             "chunk_f16_ffma2": 80000, "chunk_bf16_ffma2": 80000, "chunk_f16_mixed": 80000,
-            "ldg128_l1": 20000, "gather4": 2000, "gather8": 2000, "gather8_ffma": 2000, "alu": 20000}
+            "ldg128_l1": 20000, "gather4": 2000, "gather8": 2000, "gather8_ffma": 2000, "alu": 20000,
+            "ldg256_l1": 20000}
     res = {}
     for name in dcn._binding.PROBES:
         n = max(1, int(reps[name] * reps_scale))
@@ -717,6 +718,12 @@ def run_ceilings(reps_scale: float) -> None:
     lds = res["lds128"]["per_sm_per_clk"]
     tap_bytes = samples * 4 * si.DCNV4_P4.C * 2
     res["p4_corner_bytes_floor_us"] = round(tap_bytes / (sms * lds * clk_mhz * 1e6) * 1e6, 2)
+    # Sparse4D forward: every (unit, scale) tap reads four fp32 rows of G*C channels through L1
+    a = si.SPARSE4D
+    agg_bytes = a.samples // a.G * 4 * a.G * a.C * 4
+    for name in ("ldg128_l1", "ldg256_l1"):
+        r = res[name]["per_sm_per_clk"]
+        res[f"sparse4d_corner_bytes_floor_us_{name}"] = round(agg_bytes / (sms * r * clk_mhz * 1e6) * 1e6, 2)
     for name, v in res.items():
         if isinstance(v, dict):
             extra = f"   P4 floor {v['p4_floor_us']} us" if "p4_floor_us" in v else ""

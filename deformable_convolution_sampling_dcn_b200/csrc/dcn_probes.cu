@@ -41,7 +41,8 @@ enum Probe : int {
     kGather8 = 10,      // 8 lanes per item, 2 loads per tap (A|B as one 128-byte row), paired FMAs
     kGather8Ffma = 11,  // as kGather8 with scalar FMAs
     kAlu = 12,          // lop3.b32 (integer pipe)
-    kNumProbes = 13
+    kLdg256L1 = 13,     // 32-byte global loads (ld.global.nc.v8.f32) that hit L1
+    kNumProbes = 14
 };
 
 // Work units per thread per repetition, and their name.
@@ -54,12 +55,13 @@ __host__ __device__ constexpr double units_per_rep(int p) {
          : p == kLdg128L1 ? 8.0 * 16.0        // bytes
          : p == kGather4 ? 9.0 / 4.0          // samples (9 taps, 4 lanes per item)
          : p <= kGather8Ffma ? 9.0 / 8.0      // samples (9 taps, 8 lanes per item)
+         : p == kLdg256L1 ? 8.0 * 32.0        // bytes
          : 16.0;                              // ALU ops
 }
 
 const char *unit_name(int p) {
     switch (p) {
-        case kLds128: case kLdg128L1: return "bytes";
+        case kLds128: case kLdg128L1: case kLdg256L1: return "bytes";
         case kFfma: case kFfma2: return "fma";
         case kGather4: case kGather8: case kGather8Ffma: return "samples";
         case kAlu: return "alu ops";
@@ -235,6 +237,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             o += 512;
         }
+    } else if (P == kLdg256L1) {
+        const unsigned char *src = reinterpret_cast<const unsigned char *>(gsrc);
+        uint32_t o = (uint32_t)(threadIdx.x * 32) & (kL1Bytes - 1);
+        for (int r = 0; r < reps; ++r) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float v[8];
+                asm volatile("ld.global.nc.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                             : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]),
+                               "=f"(v[7])
+                             : "l"(src + ((o + j * 4096) & (kL1Bytes - 1))));
+                sink ^= __float_as_uint(v[0]) ^ __float_as_uint(v[7]);
+            }
+            o += 1024;
+        }
     } else if (P == kGather4) {
         const int gi = lane >> 2, q = lane & 3;
         const uint32_t bq = sbase + q * 16;
@@ -366,6 +383,7 @@ extern "C" dcn_status dcn_probe_rate(int32_t probe, int32_t reps, void *dev_buf,
         case kGather8: e = launch_probe<kGather8>(reps, sms, res, src, st); break;
         case kGather8Ffma: e = launch_probe<kGather8Ffma>(reps, sms, res, src, st); break;
         case kAlu: e = launch_probe<kAlu>(reps, sms, res, src, st); break;
+        case kLdg256L1: e = launch_probe<kLdg256L1>(reps, sms, res, src, st); break;
     }
     if (e != cudaSuccess) return DCN_ERR_CUDA;
     *units_per_cta = units_per_rep(probe) * (double)kThreads * (double)reps;

@@ -243,6 +243,162 @@ __global__ void __launch_bounds__(kAggWarps * 32) agg_forward_pairs_f32(AggArgs 
     if (dirty) flush();
 }
 
+// fp32 forward with the tap decode shared by the warp.  Warp w takes units
+// [U*w/NW, U*(w+1)/NW) (unit = (b*A + anchor)*P*cams + point*cams + camera,
+// so consecutive units mostly share an anchor).  The (unit, scale) taps of a
+// batch of 32 / S units are decoded one per lane (location, table entry,
+// floor, the four corner rows and their bilinear weights); the lanes then walk
+// the batch's taps together, taking each tap's rows and weights by shuffle,
+// so the decode runs once per tap instead of once per lane.  Each unit's
+// scales are unrolled so that their corner loads are in flight together.  The
+// partial row of an anchor is added to the zeroed output when the next unit
+// belongs to another anchor.
+// A lane holds VW consecutive channels per load: VW = 8 (one 32-byte load,
+// sm_100's ld.global.v8.f32) where the group width C allows it, else 4.
+// Needs S <= 32, fewer than 2^31 units and B*num_rows < 2^31.
+__device__ __forceinline__ void ldg_v(const float *p, float (&v)[8]) {
+    asm volatile("ld.global.nc.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+                 : "l"(p));
+}
+__device__ __forceinline__ void ldg_v(const float *p, float (&v)[4]) {
+    const float4 t = __ldg(reinterpret_cast<const float4 *>(p));
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+}
+
+template <int CPL, int VW>
+__global__ void __launch_bounds__(kAggWarps * 32) agg_forward_coop_f32(AggArgs a, long long units, int total_warps) {
+    constexpr int V = VW;                  // channels per lane and load
+    constexpr int NL = CPL * 4 / VW;       // loads per lane and corner row
+    constexpr int ROW = CPL * 32 * 4;      // channels of a row
+    __shared__ int4 tab[kAggTableMax];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int S = a.scales;
+    const int CS = a.cams * S;
+    const bool tab_smem = CS <= kAggTableMax;
+    if (tab_smem)
+        for (int i = threadIdx.x; i < CS; i += blockDim.x) tab[i] = load_table(a, i);
+    __syncthreads();
+
+    const int NB = 32 / S;                              // units per batch
+    const int my_bu = lane / S, my_s = lane - my_bu * S;  // this lane's tap of a batch
+    const int gw = blockIdx.x * kAggWarps + warp;
+    const long long p0 = units * gw / total_warps, p1 = units * (gw + 1) / total_warps;
+    const int pairs = a.P * a.cams;
+    const float *__restrict__ wts = static_cast<const float *>(a.weights);
+    const float *__restrict__ feat = static_cast<const float *>(a.feat);
+    const float2 *__restrict__ locp = reinterpret_cast<const float2 *>(a.loc);
+    float *__restrict__ out = static_cast<float *>(a.out);
+    int grp[NL];
+#pragma unroll
+    for (int j = 0; j < NL; ++j) grp[j] = (32 * j + lane) * V / a.C;
+    float acc[NL][V];
+#pragma unroll
+    for (int j = 0; j < NL; ++j)
+#pragma unroll
+        for (int v = 0; v < V; ++v) acc[j][v] = 0.0f;
+    bool nan_acc = false;
+    int cur_ba = -1;  // anchor (b*A + a) whose partial row acc holds
+
+    for (long long pb = p0; pb < p1; pb += NB) {
+        const int nb = (int)min((long long)NB, p1 - pb);
+        // ---- decode: lane = (unit my_bu, scale my_s) of this batch
+        const bool tv = my_bu < nb;
+        int uid = 0;
+        if (tv) uid = (int)(pb + my_bu);
+        const int ba = uid / pairs;
+        const int cam = (uid - ba * pairs) % a.cams;
+        const int b = ba / a.A;
+        const float2 uv = tv ? __ldg(locp + uid) : make_float2(0.0f, 0.0f);
+        const int4 t = tab_smem ? tab[cam * S + my_s] : load_table(a, cam * S + my_s);
+        Tap tp{0, 0, 0.0f, 0.0f};
+        int st = make_tap(fmaf(uv.y, (float)t.x, -0.5f), fmaf(uv.x, (float)t.y, -0.5f), t.x, t.y, tp);
+        if (!tv) st = 0;
+        const unsigned nanm = __ballot_sync(0xffffffffu, st < 0);
+        int rw[4];
+        float gw4[4];
+        const long long row00 = (long long)t.z + (long long)tp.y0 * t.y + tp.x0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int y = tp.y0 + (c >> 1), x = tp.x0 + (c & 1);
+            const long long row = row00 + (c >> 1) * t.y + (c & 1);
+            const bool ok = st > 0 && (unsigned)y < (unsigned)t.x && (unsigned)x < (unsigned)t.y &&
+                            (unsigned long long)row < (unsigned long long)a.rows;
+            rw[c] = ok ? (int)((long long)b * a.rows + row) : -1;
+            gw4[c] = ok ? ((c >> 1) ? tp.ly : 1.0f - tp.ly) * ((c & 1) ? tp.lx : 1.0f - tp.lx) : 0.0f;
+        }
+        // ---- sample: every lane, every tap of the batch
+        for (int bu = 0; bu < nb; ++bu) {
+            const int kb = bu * S;
+            const int ba_k = __shfl_sync(0xffffffffu, ba, kb);
+            const int uid_k = __shfl_sync(0xffffffffu, uid, kb);
+            if (ba_k != cur_ba) {
+                if (cur_ba >= 0) {
+                    float *o = out + (long long)cur_ba * ROW + lane * V;
+#pragma unroll
+                    for (int j = 0; j < NL; ++j) {
+                        if (nan_acc) {
+#pragma unroll
+                            for (int v = 0; v < V; ++v) acc[j][v] = __int_as_float(0x7fc00000);
+                        }
+#pragma unroll
+                        for (int h = 0; h < V; h += 4) red_add16<float>(o + 32 * j * V + h, acc[j] + h);
+#pragma unroll
+                        for (int v = 0; v < V; ++v) acc[j][v] = 0.0f;
+                    }
+                    nan_acc = false;
+                }
+                cur_ba = ba_k;
+            }
+            const unsigned um = S == 32 ? 0xffffffffu : ((1u << S) - 1u) << kb;
+            nan_acc |= (nanm & um) != 0;
+            const float *wu = wts + (long long)uid_k * S * a.G;
+#pragma unroll 4
+            for (int s = 0; s < S; ++s) {
+                const int k = kb + s;
+                float w[NL];
+#pragma unroll
+                for (int j = 0; j < NL; ++j) w[j] = __ldg(wu + s * a.G + grp[j]);
+                float g[4];
+                float f[4][NL][V];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int r = __shfl_sync(0xffffffffu, rw[c], k);
+                    g[c] = __shfl_sync(0xffffffffu, gw4[c], k);
+                    const float *src = feat + (long long)(r < 0 ? 0 : r) * ROW + lane * V;
+#pragma unroll
+                    for (int j = 0; j < NL; ++j) {
+#pragma unroll
+                        for (int v = 0; v < V; ++v) f[c][j][v] = 0.0f;
+                        if (r >= 0) ldg_v(src + 32 * j * V, f[c][j]);
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int j = 0; j < NL; ++j) {
+                        const float wg = w[j] * g[c];
+#pragma unroll
+                        for (int v = 0; v < V; ++v) acc[j][v] = fmaf(wg, f[c][j][v], acc[j][v]);
+                    }
+            }
+        }
+    }
+    if (cur_ba >= 0) {
+        float *o = out + (long long)cur_ba * ROW + lane * V;
+#pragma unroll
+        for (int j = 0; j < NL; ++j) {
+            if (nan_acc) {
+#pragma unroll
+                for (int v = 0; v < V; ++v) acc[j][v] = __int_as_float(0x7fc00000);
+            }
+#pragma unroll
+            for (int h = 0; h < V; h += 4) red_add16<float>(o + 32 * j * V + h, acc[j] + h);
+        }
+    }
+}
+
 // Backward with pair-granular persistent work (every storage type): warp w
 // of the grid owns the contiguous (anchor, pair) units [U*w/NW, U*(w+1)/NW),
 // so every warp has the same number of samples whatever the anchor count.
@@ -386,6 +542,32 @@ __global__ void __launch_bounds__(kAggWarps * 32) agg_backward_pairs(AggArgs a, 
     }
 }
 
+template <int CPL, int VW>
+cudaError_t launch_coop_k(const AggArgs &a, cudaStream_t stream) {
+    int dev = 0, sms = 148, per_sm = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, agg_forward_coop_f32<CPL, VW>, kAggWarps * 32, 0);
+    if (per_sm < 1) per_sm = 1;
+    const long long units = (long long)a.B * a.A * a.P * a.cams;
+    long long ctas = (long long)sms * per_sm;
+    if (ctas * kAggWarps > units) ctas = (units + kAggWarps - 1) / kAggWarps;
+    cudaError_t e = cudaMemsetAsync(a.out, 0, (size_t)a.B * a.A * a.G * a.C * sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+    agg_forward_coop_f32<CPL, VW><<<(unsigned)ctas, kAggWarps * 32, 0, stream>>>(a, units, (int)(ctas * kAggWarps));
+    return cudaGetLastError();
+}
+
+template <int CPL>
+cudaError_t launch_coop(const AggArgs &a, cudaStream_t stream) {
+    // 32-byte loads need 8 channels of one group per lane and a 32-byte aligned
+    // feat (the ABI guarantees 16; rows are multiples of 32 bytes)
+    constexpr int VW8 = CPL % 2 == 0 ? 8 : 4;
+    if (CPL % 2 == 0 && a.C % 8 == 0 && (reinterpret_cast<uintptr_t>(a.feat) & 31) == 0)
+        return launch_coop_k<CPL, VW8>(a, stream);
+    return launch_coop_k<CPL, 4>(a, stream);
+}
+
 template <typename T, int CPL>
 cudaError_t launch(const AggArgs &a, bool bwd, cudaStream_t stream) {
     const unsigned grid = (unsigned)((long long)a.B * a.A);
@@ -401,6 +583,9 @@ cudaError_t launch(const AggArgs &a, bool bwd, cudaStream_t stream) {
         long long ctas = (long long)sms * per_sm;
         if (ctas * kAggWarps > units) ctas = (units + kAggWarps - 1) / kAggWarps;
         agg_backward_pairs<T, CPL><<<(unsigned)ctas, kAggWarps * 32, 0, stream>>>(a, units, (int)(ctas * kAggWarps));
+    } else if (sizeof(T) == 4 && a.scales <= 32 && (long long)a.B * a.A * a.P * a.cams <= 0x7fffffffLL &&
+               (long long)a.B * a.rows <= 0x7fffffffLL) {
+        return launch_coop<CPL>(a, stream);
     } else if (sizeof(T) == 4) {
         // fp32 output: pair-granular persistent warps, partial rows added in L2
         int dev = 0, sms = 148, per_sm = 1;

@@ -16,6 +16,7 @@ def run_fwd(inp, dev):
     keys = ("feat", "spatial_shape", "scale_start_index", "sampling_location", "weights")
     out = d.deform_agg_forward(*(inp[k].to(dev) for k in keys))
     torch.cuda.synchronize()
+    assert d.lib().dcn_take_device_error() == 0
     ref = oracle.agg_forward(*(inp[k] for k in keys))
     return out, ref
 
@@ -43,6 +44,40 @@ def test_sparse4d_full_size(cuda_dev):
     out, ref = run_fwd(inp, cuda_dev)
     r = assert_close_fwd(out, ref, "sparse4d")
     print(f"sparse4d: worst err/bound {r:.3f}")
+
+
+def test_feat_only_16_byte_aligned(cuda_dev):
+    """A feat that is 16- but not 32-byte aligned takes the 16-byte loads."""
+    import deformable_convolution_sampling_dcn_b200 as d
+
+    shape = si.AggShape(B=2, num_cams=3, scales=((9, 13), (4, 6)), num_anchors=21, num_pts=4, G=8, C=32)
+    inp = si.agg_inputs(shape, 516, loc_lo=-0.1, loc_hi=1.1)
+    f = inp["feat"]
+    buf = torch.empty(f.numel() + 4, dtype=f.dtype, device=cuda_dev)
+    feat = buf[4:].view(f.shape)
+    feat.copy_(f.to(cuda_dev))
+    assert feat.data_ptr() % 32 == 16
+    keys = ("spatial_shape", "scale_start_index", "sampling_location", "weights")
+    out = d.deform_agg_forward(feat, *(inp[k].to(cuda_dev) for k in keys))
+    torch.cuda.synchronize()
+    ref = oracle.agg_forward(*(inp[k] for k in ("feat",) + keys))
+    assert_close_fwd(out, ref, "16-byte aligned feat")
+
+
+def test_nan_and_far_locations(cuda_dev):
+    """NaN locations make their anchor's row NaN; locations far outside [0, 1]
+    contribute zero."""
+    shape = si.AggShape(B=2, num_cams=3, scales=((9, 13), (4, 6)), num_anchors=21, num_pts=4, G=4, C=32)
+    inp = si.agg_inputs(shape, 515, loc_lo=-0.1, loc_hi=1.1)
+    loc = inp["sampling_location"]
+    loc[0, 3, 1, 2, 0] = float("nan")
+    loc[1, 7, 0, 0, 1] = float("nan")
+    loc[0, 5, 2, 1] = torch.tensor([-40.0, 3.0])
+    loc[1, 11, 3, 2] = torch.tensor([float("inf"), -float("inf")])
+    loc[1, 12, 0, 1] = torch.tensor([2.0e9, 0.5])
+    out, ref = run_fwd(inp, cuda_dev)
+    assert np.isnan(ref).sum() == 2 * shape.G * shape.C
+    assert_close_fwd(out, ref, "nan/far")
 
 
 SMALL = [
