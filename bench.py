@@ -700,7 +700,7 @@ def run_ceilings(reps_scale: float) -> None:
     reps = {"lds128": 20000, "chunk_f32_ffma2": 80000, "ffma": 20000, "ffma2": 20000, "chunk_f16_ffma": 80000,
             "chunk_f16_ffma2": 80000, "chunk_bf16_ffma2": 80000, "chunk_f16_mixed": 80000,
             "ldg128_l1": 20000, "gather4": 2000, "gather8": 2000, "gather8_ffma": 2000, "alu": 20000,
-            "ldg256_l1": 20000}
+            "ldg256_l1": 20000, "atoms_f32": 20000}
     res = {}
     for name in dcn._binding.PROBES:
         n = max(1, int(reps[name] * reps_scale))

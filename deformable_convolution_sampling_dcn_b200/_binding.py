@@ -164,7 +164,8 @@ def take_device_error() -> int:
 
 
 PROBES = ("lds128", "chunk_f32_ffma2", "ffma", "ffma2", "chunk_f16_ffma", "chunk_f16_ffma2", "chunk_bf16_ffma2",
-          "chunk_f16_mixed", "ldg128_l1", "gather4", "gather8", "gather8_ffma", "alu", "ldg256_l1")
+          "chunk_f16_mixed", "ldg128_l1", "gather4", "gather8", "gather8_ffma", "alu", "ldg256_l1",
+          "atoms_f32")
 
 
 def probe_rate(name: str, reps: int, device=None) -> Tuple[float, str]:

@@ -165,6 +165,9 @@ __global__ void __launch_bounds__(kStagedMaxThreads, 1)
     const int K = a.kh * a.kw;
     const int GC = a.G * a.C;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // a programmatic dependent on the stream (the projection GEMM) may launch
+    // now; it waits for this grid's completion before reading its output
+    asm volatile("griddepcontrol.launch_dependents;");
 
     extern __shared__ __align__(1024) unsigned char smem[];
     // [band 0][band 1 if nbuf == 2][rec weights: NC x KMAX x IPW float4][rec addrs: NC x KMAX x IPW int2]

@@ -42,7 +42,8 @@ enum Probe : int {
     kGather8Ffma = 11,  // as kGather8 with scalar FMAs
     kAlu = 12,          // lop3.b32 (integer pipe)
     kLdg256L1 = 13,     // 32-byte global loads (ld.global.nc.v8.f32) that hit L1
-    kNumProbes = 14
+    kAtomsF32 = 14,     // red.shared.add.f32, a warp's 32 lanes on 32 distinct banks
+    kNumProbes = 15
 };
 
 // Work units per thread per repetition, and their name.
@@ -56,6 +57,7 @@ __host__ __device__ constexpr double units_per_rep(int p) {
          : p == kGather4 ? 9.0 / 4.0          // samples (9 taps, 4 lanes per item)
          : p <= kGather8Ffma ? 9.0 / 8.0      // samples (9 taps, 8 lanes per item)
          : p == kLdg256L1 ? 8.0 * 32.0        // bytes
+         : p == kAtomsF32 ? 8.0               // shared-memory fp32 reductions
          : 16.0;                              // ALU ops
 }
 
@@ -65,6 +67,7 @@ const char *unit_name(int p) {
         case kFfma: case kFfma2: return "fma";
         case kGather4: case kGather8: case kGather8Ffma: return "samples";
         case kAlu: return "alu ops";
+        case kAtomsF32: return "shared reductions";
         default: return "chunks";
     }
 }
@@ -252,6 +255,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             o += 1024;
         }
+    } else if (P == kAtomsF32) {
+        uint32_t a = sbase + (uint32_t)(warp * 512 + lane * 4);
+        for (int r = 0; r < reps; ++r) {
+            const float v = __int_as_float(0x3f800000 | (r & 0xff));
+#pragma unroll
+            for (int j = 0; j < 8; ++j) asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(a + j * 8192), "f"(v) : "memory");
+            a ^= 4096;
+        }
     } else if (P == kGather4) {
         const int gi = lane >> 2, q = lane & 3;
         const uint32_t bq = sbase + q * 16;
@@ -384,6 +395,7 @@ extern "C" dcn_status dcn_probe_rate(int32_t probe, int32_t reps, void *dev_buf,
         case kGather8Ffma: e = launch_probe<kGather8Ffma>(reps, sms, res, src, st); break;
         case kAlu: e = launch_probe<kAlu>(reps, sms, res, src, st); break;
         case kLdg256L1: e = launch_probe<kLdg256L1>(reps, sms, res, src, st); break;
+        case kAtomsF32: e = launch_probe<kAtomsF32>(reps, sms, res, src, st); break;
     }
     if (e != cudaSuccess) return DCN_ERR_CUDA;
     *units_per_cta = units_per_rep(probe) * (double)kThreads * (double)reps;

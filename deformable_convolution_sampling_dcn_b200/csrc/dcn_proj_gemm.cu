@@ -119,27 +119,27 @@ __global__ void __launch_bounds__(kGThreads, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // The launcher makes this kernel a programmatic dependent of the core kernel
+    // that writes the pixel matrix, so it may start while that kernel's last CTAs
+    // run: the producer issues this CTA's weight rows (which the core kernel does
+    // not write) first, then every thread waits for the core kernel to complete
+    // before any wait of its own starts (the instruction returns at once when the
+    // launch was an ordinary one).
+    int wissued = 0;  // weight K-blocks issued (producer thread)
+    if (warp == 0 && lane == 0 && pt0 < p.PT)
+        for (int j = 0; j < KB; ++j, ++wissued) {
+            mbar_arrive_expect_tx(wfull + 8 * j, (uint32_t)wblk);
+            tma_load_2d(smem_u32(wres + j * wblk), &bmap, wfull + 8 * j, j * kBK, nt * p.BN);
+        }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     if (warp == 0) {
-        // ---- producer: this CTA's weight rows once, then the pixel K-blocks of its tiles
+        // ---- producer: the pixel K-blocks of this CTA's tiles
         if (lane == 0) {
             uint32_t s = 0, pass = 0;
             long long issued = 0;
-            int wissued = 0;  // weight K-blocks issued
-            bool first = true;
-            for (long long pt = pt0; pt < p.PT && !*abort_flag; pt += pstep, first = false) {
+            for (long long pt = pt0; pt < p.PT && !*abort_flag; pt += pstep) {
                 for (int kb = 0; kb < KB; ++kb) {
-                    // first tile: weight K-block kb just ahead of pixel K-block kb while the ring
-                    // fills, then every remaining weight K-block at once
-                    if (first && kb < kGStages) {
-                        mbar_arrive_expect_tx(wfull + 8 * kb, (uint32_t)wblk);
-                        tma_load_2d(smem_u32(wres + kb * wblk), &bmap, wfull + 8 * kb, kb * kBK, nt * p.BN);
-                        ++wissued;
-                    }
-                    if (first && kb == kGStages)
-                        for (int j = kGStages; j < KB; ++j, ++wissued) {
-                            mbar_arrive_expect_tx(wfull + 8 * j, (uint32_t)wblk);
-                            tma_load_2d(smem_u32(wres + j * wblk), &bmap, wfull + 8 * j, j * kBK, nt * p.BN);
-                        }
                     if (pass >= 1 && !wait_or_abort(empty0 + 8 * s, (pass - 1) & 1, abort_flag)) {
                         raise_abort(abort_flag, p.err);
                         break;
@@ -312,8 +312,19 @@ cudaError_t launch_t(const void *core, const void *weight, const void *bias, voi
     auto kern = proj_gemm_kernel<T>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<p.n_cta, kGThreads, smem, stream>>>(amap, bmap, p);
-    return cudaGetLastError();
+    // programmatic dependent launch: the CTAs may start (and fetch their weight
+    // rows) as the preceding kernel on the stream finishes
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.n_cta);
+    cfg.blockDim = dim3(kGThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, amap, bmap, p);
 }
 
 }  // namespace

@@ -542,6 +542,13 @@ __global__ void __launch_bounds__(kAggWarps * 32) agg_backward_pairs(AggArgs a, 
     }
 }
 
+// Shapes the warp-shared tap decode takes: one tap per lane needs S <= 32;
+// unit and row indices travel as int32.
+bool coop_fits(const AggArgs &a) {
+    return a.scales <= 32 && (long long)a.B * a.A * a.P * a.cams <= 0x7fffffffLL &&
+           (long long)a.B * a.rows <= 0x7fffffffLL;
+}
+
 template <int CPL, int VW>
 cudaError_t launch_coop_k(const AggArgs &a, cudaStream_t stream) {
     int dev = 0, sms = 148, per_sm = 1;
@@ -583,8 +590,7 @@ cudaError_t launch(const AggArgs &a, bool bwd, cudaStream_t stream) {
         long long ctas = (long long)sms * per_sm;
         if (ctas * kAggWarps > units) ctas = (units + kAggWarps - 1) / kAggWarps;
         agg_backward_pairs<T, CPL><<<(unsigned)ctas, kAggWarps * 32, 0, stream>>>(a, units, (int)(ctas * kAggWarps));
-    } else if (sizeof(T) == 4 && a.scales <= 32 && (long long)a.B * a.A * a.P * a.cams <= 0x7fffffffLL &&
-               (long long)a.B * a.rows <= 0x7fffffffLL) {
+    } else if (sizeof(T) == 4 && coop_fits(a)) {
         return launch_coop<CPL>(a, stream);
     } else if (sizeof(T) == 4) {
         // fp32 output: pair-granular persistent warps, partial rows added in L2

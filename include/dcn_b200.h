@@ -327,6 +327,7 @@ dcn_status dcn_selftest_bounded_wait(int32_t limit_us, dcn_stream_t stream);
  *   11  gather, 8 lanes per item, FMAs (samples)
  *   12  integer lop3 (ops)
  *   13  32-byte global loads (ld.global.nc.v8.f32) hitting L1 (bytes)
+ *   14  red.shared.add.f32, 32 distinct banks per warp (shared reductions)
  * dev_buf is a caller-owned device buffer of at least 36,864 bytes, 256-byte
  * aligned: on completion its first two 64-bit words hold the sum over the
  * CTAs of their SM-clock cycles and the number of CTAs (the rest is scratch
