@@ -325,7 +325,12 @@ dcn_status dcn_core_backward(const dcn_params *p, const void *x, const void *off
     dcnb::CoreArgs a = core_args(p, Ho, Wo);
     a.x = x; a.offset = offset; a.mask = mask; a.grad_out = grad_out;
     a.grad_x = grad_x; a.grad_offset = grad_offset; a.grad_mask = grad_mask;
-    return cuda_status(dcnb::launch_core_backward_generic(a, (cudaStream_t)stream), "dcn_core_backward launch");
+    bool handled = false;
+    cudaError_t e = cudaSuccess;
+    const char *force = getenv("DCN_B200_FORCE_GENERIC");
+    if (!(force && force[0] == '1')) e = dcnb::launch_core_backward_staged(a, (cudaStream_t)stream, &handled);
+    if (!handled) e = dcnb::launch_core_backward_generic(a, (cudaStream_t)stream);
+    return cuda_status(e, "dcn_core_backward launch");
 }
 
 dcn_status deform_agg_forward(const dagg_params *p, const void *feat, const int32_t *spatial_shape,

@@ -65,6 +65,9 @@ struct RoiArgs {
 // cudaGetLastError() of the launch.
 cudaError_t launch_core_forward_generic(const CoreArgs &a, cudaStream_t stream);
 cudaError_t launch_core_backward_generic(const CoreArgs &a, cudaStream_t stream);
+// Staged backward (TMA row bands, per-tap records) for fp32 storage with 128-byte
+// groups and K <= 9; *handled stays false for other shapes.
+cudaError_t launch_core_backward_staged(const CoreArgs &a, cudaStream_t stream, bool *handled);
 // Shared-memory path; sets *handled = false (and launches nothing) when the
 // problem does not fit it.
 cudaError_t launch_core_forward_plane(const CoreArgs &a, cudaStream_t stream, bool *handled);

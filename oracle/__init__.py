@@ -63,6 +63,8 @@ def _bind(lib):
     lib.oracle_dcn_forward.restype = None
     lib.oracle_dcn_backward.argtypes = [i] * 13 + [ctypes.c_float, i, dp, dp, dp, dp, dp, dp, dp]
     lib.oracle_dcn_backward.restype = None
+    lib.oracle_dcn_grad_x_budget.argtypes = [i] * 13 + [ctypes.c_float, i, dp, dp, dp, dp, dp]
+    lib.oracle_dcn_grad_x_budget.restype = None
     lib.oracle_agg_forward.argtypes = [i] * 8 + [dp, ip, ip, fp, dp, dp]
     lib.oracle_agg_forward.restype = None
     lib.oracle_agg_backward.argtypes = [i] * 8 + [dp, ip, ip, fp, dp, dp, dp, dp, dp]
@@ -179,6 +181,24 @@ def dcn_backward(x, offset, mask, grad_out, *, G: int, kh: int = 3, kw: int = 3,
                             _ptr(go, ctypes.c_double), _ptr(gx, ctypes.c_double),
                             _ptr(goff, ctypes.c_double), _ptr(gm, ctypes.c_double))
     return {"grad_x": gx, "grad_offset": goff, "grad_mask": gm}
+
+
+def dcn_grad_x_budget(offset, mask, grad_out, *, x_shape, G: int, kh: int = 3, kw: int = 3, stride=(1, 1),
+                      pad=(1, 1), dil=(1, 1), offset_scale: float = 1.0, softmax: bool = False,
+                      lib=None) -> Dict[str, np.ndarray]:
+    """Per grad_x element: the absolute sum of its contributions (abs_sum,
+    [B,H,W,G*C]) and their number (terms, [B,H,W,G]); see dcn_oracle.c."""
+    lib = lib or load()
+    offset, mask, go = _f64(offset), _f64(mask), _f64(grad_out)
+    B, H, W, GC = x_shape
+    C = GC // G
+    abs_sum = np.empty((B, H, W, GC), dtype=np.float64)
+    terms = np.empty((B, H, W, G), dtype=np.float64)
+    lib.oracle_dcn_grad_x_budget(B, H, W, G, C, kh, kw, stride[0], stride[1], pad[0], pad[1], dil[0], dil[1],
+                                 float(offset_scale), int(bool(softmax)), _ptr(offset, ctypes.c_double),
+                                 _ptr(mask, ctypes.c_double), _ptr(go, ctypes.c_double),
+                                 _ptr(abs_sum, ctypes.c_double), _ptr(terms, ctypes.c_double))
+    return {"abs_sum": abs_sum, "terms": terms}
 
 
 def _agg_common(feat, spatial_shape, scale_start_index, sampling_location, weights):

@@ -342,6 +342,68 @@ void oracle_dcn_backward(int B, int H, int W, int G, int C, int kh, int kw,
 }
 
 /*
+ * Error budget of an input gradient summed by atomic additions: for every
+ * grad_x element, the sum of the absolute values of its contributions
+ * |m_k G(q,p) grad_out_c| (abs_sum, [B,H,W,G*C]) and how many contributions it
+ * receives (terms, [B,H,W,G], the same for every channel of a group).  When a
+ * device adds the contributions one by one in a storage precision with unit
+ * roundoff u, each partial sum and each contribution is rounded once, and the
+ * recursive-summation bound (Higham, "Accuracy and Stability of Numerical
+ * Algorithms", 2nd ed., section 4.2) limits the error of the stored result to
+ * gamma_(n+1) * abs_sum, gamma_m = m u / (1 - m u), n = terms: whatever the
+ * order in which the atomics land.  The taps are enumerated exactly as in
+ * oracle_dcn_backward.
+ */
+void oracle_dcn_grad_x_budget(int B, int H, int W, int G, int C, int kh, int kw,
+                              int sh, int sw, int ph, int pw, int dh, int dw,
+                              float offset_scale, int softmax,
+                              const double *offset, const double *mask, const double *grad_out,
+                              double *abs_sum, double *terms)
+{
+    const int K = kh * kw;
+    const int Ho = (H + 2 * ph - (dh * (kh - 1) + 1)) / sh + 1;
+    const int Wo = (W + 2 * pw - (dw * (kw - 1) + 1)) / sw + 1;
+    memset(abs_sum, 0, sizeof(double) * (size_t)B * H * W * G * C);
+    memset(terms, 0, sizeof(double) * (size_t)B * H * W * G);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int g = 0; g < G; ++g) {
+            double *m = (double *)malloc(sizeof(double) * (size_t)K);
+            for (int ho = 0; ho < Ho; ++ho)
+                for (int wo = 0; wo < Wo; ++wo) {
+                    const size_t item = (((size_t)b * Ho + ho) * Wo + wo) * G + g;
+                    const double *go = grad_out + item * C;
+                    modulation(mask + item * K, K, softmax, m);
+                    for (int i = 0; i < kh; ++i)
+                        for (int j = 0; j < kw; ++j) {
+                            const int k = i * kw + j;
+                            const int by = ho * sh - ph + i * dh;
+                            const int bx = wo * sw - pw + j * dw;
+                            const double *d = offset + (item * K + k) * 2;
+                            const float px = fmaf(offset_scale, (float)d[0], (float)bx);
+                            const float py = fmaf(offset_scale, (float)d[1], (float)by);
+                            if (isnan(px) || isnan(py)) continue;
+                            const double fy = floor((double)py), fx = floor((double)px);
+                            if (!(fy >= -1.0 && fy <= H - 1 && fx >= -1.0 && fx <= W - 1)) continue;
+                            const int y0 = (int)fy, x0 = (int)fx;
+                            for (int qy = y0; qy <= y0 + 1; ++qy) {
+                                if (qy < 0 || qy >= H) continue;
+                                for (int qx = x0; qx <= x0 + 1; ++qx) {
+                                    if (qx < 0 || qx >= W) continue;
+                                    const double Gq = g_kernel(qx, px) * g_kernel(qy, py);
+                                    const size_t pixel = ((size_t)b * H + qy) * W + qx;
+                                    double *aq = abs_sum + pixel * (size_t)G * C + (size_t)g * C;
+                                    for (int c = 0; c < C; ++c) aq[c] += fabs(m[k] * Gq * go[c]);
+                                    terms[pixel * G + g] += 1.0;
+                                }
+                            }
+                        }
+                }
+            free(m);
+        }
+}
+
+/*
  * Multi-camera multi-scale deformable aggregation, forward.
  *   feat    [B, rows, G*C]; camera cam, scale s occupies rows
  *           start[cam*S + s] + y*W_s + x for its H_s x W_s map

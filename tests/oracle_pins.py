@@ -472,7 +472,63 @@ def pin_backward_right_derivative_at_minus_one(lib):
         assert abs(an - fd) <= 1e-9 * (1 + abs(fd)), f"right derivative at p = -1: {an} vs {fd}"
 
 
-BACKWARD_PINS = [pin_backward_fd, pin_backward_autograd, pin_backward_right_derivative_at_minus_one]
+def pin_grad_x_budget(lib):
+    """The error budget of grad_x: per element, the number of contributions and
+    the sum of their absolute values, by brute force over every (item, point,
+    corner) with positions formed in fp32; and, for non-negative modulation and
+    grad_out (no cancellation), the absolute sum is the oracle's grad_x itself."""
+    B, G, C = 2, 2, 3
+    for softmax in (False, True):
+        for geom in GEOMS[:4]:
+            H, W, kh, kw, stride, pad, dil = geom
+            x, off, mask = rand_case(411, B, H, W, G, C, kh, kw, stride, pad, dil, 1.5, quant=2.0 ** -10)
+            Ho, Wo = oracle.out_hw(H, W, kh, kw, *stride, *pad, *dil)
+            rng = np.random.default_rng(412)
+            go = rng.standard_normal((B, Ho, Wo, G * C))
+            s = 0.75
+            bud = oracle.dcn_grad_x_budget(off, mask, go, x_shape=x.shape, G=G, kh=kh, kw=kw, stride=stride,
+                                           pad=pad, dil=dil, offset_scale=s, softmax=softmax, lib=lib)
+            py, px = positions32(off, Ho, Wo, kh, kw, stride, pad, dil, s)
+            K = kh * kw
+            if softmax:
+                e = np.exp(mask - mask.max(axis=-1, keepdims=True))
+                m = e / e.sum(axis=-1, keepdims=True)
+            else:
+                m = mask
+            A = np.zeros((B, H, W, G * C))
+            n = np.zeros((B, H, W, G))
+            for b in range(B):
+                for ho in range(Ho):
+                    for wo in range(Wo):
+                        for g in range(G):
+                            for k in range(K):
+                                yy, xx = py[b, ho, wo, g, k], px[b, ho, wo, g, k]
+                                y0, x0 = int(np.floor(yy)), int(np.floor(xx))
+                                for qy in (y0, y0 + 1):
+                                    for qx in (x0, x0 + 1):
+                                        if not (0 <= qy < H and 0 <= qx < W):
+                                            continue
+                                        wgt = max(0.0, 1 - abs(qx - xx)) * max(0.0, 1 - abs(qy - yy))
+                                        if wgt == 0.0:
+                                            continue
+                                        gsl = slice(g * C, (g + 1) * C)
+                                        A[b, qy, qx, gsl] += np.abs(m[b, ho, wo, g, k] * wgt * go[b, ho, wo, gsl])
+                                        n[b, qy, qx, g] += 1
+            assert np.allclose(bud["abs_sum"], A, rtol=1e-12, atol=1e-14), "grad_x abs_sum"
+            assert np.array_equal(bud["terms"], n), "grad_x terms"
+    # no cancellation: the absolute sum equals grad_x
+    H, W, kh, kw, stride, pad, dil = GEOMS[0]
+    x, off, mask = rand_case(413, 1, H, W, G, C, kh, kw, stride, pad, dil, 1.5, quant=2.0 ** -10)
+    Ho, Wo = oracle.out_hw(H, W, kh, kw, *stride, *pad, *dil)
+    go = np.abs(np.random.default_rng(414).standard_normal((1, Ho, Wo, G * C)))
+    mask = np.abs(mask)
+    gr = oracle.dcn_backward(x, off, mask, go, G=G, lib=lib)
+    bud = oracle.dcn_grad_x_budget(off, mask, go, x_shape=x.shape, G=G, lib=lib)
+    assert np.allclose(bud["abs_sum"], gr["grad_x"], rtol=1e-12, atol=1e-14), "abs_sum vs grad_x"
+
+
+BACKWARD_PINS = [pin_backward_fd, pin_backward_autograd, pin_backward_right_derivative_at_minus_one,
+                 pin_grad_x_budget]
 AGG_PINS = [pin_agg_brute_force, pin_agg_grid_sample, pin_agg_backward]
 ALL_PINS = CORE_PINS + BACKWARD_PINS + AGG_PINS
 

@@ -21,7 +21,13 @@ beyond fp32 summation is that one rounding (at most 2^-11 resp. 2^-8
 relative), which the 2e-3 / 8e-3 bars cover with room to spare while a few
 percent of error (a mis-scaled or dropped term) fails them.  grad_x in
 16-bit storage is summed by packed half-precision atomic adds, each rounding
-to the storage type, so it keeps the wider bars.
+to the storage type, so it keeps the wider bars; where the oracle's error
+budget is passed (`budget`: per element the absolute sum A of the n
+contributions and n itself), an element may instead stay within the
+recursive-summation bound gamma_(n+1) * A, gamma_m = m u / (1 - m u), u the
+storage type's unit roundoff (2^-24, 2^-11, 2^-8): the bound that holds for
+any order of the atomic additions, which matters where a sum cancels far
+below its terms.
 NaN must match NaN exactly.
 """
 from __future__ import annotations
@@ -63,18 +69,36 @@ def assert_close_fwd(gpu: torch.Tensor, ref: np.ndarray, what: str = "out") -> f
     return float(ratio.max())
 
 
-def assert_close_bwd(gpu: torch.Tensor, ref: np.ndarray, what: str, atomic: bool = True) -> float:
+# Unit roundoff of each storage type (round to nearest).
+UNIT_ROUNDOFF = {torch.float32: 2.0 ** -24, torch.float16: 2.0 ** -11, torch.bfloat16: 2.0 ** -8}
+
+
+def summation_bound(abs_sum: np.ndarray, terms: np.ndarray, dtype: torch.dtype) -> np.ndarray:
+    """gamma_(n+1) * A: the error bound of n contributions with absolute sum A
+    added one by one, each partial sum and each contribution rounded once."""
+    mu = (terms + 1.0) * UNIT_ROUNDOFF[dtype]
+    return mu / (1.0 - mu) * abs_sum
+
+
+def assert_close_bwd(gpu: torch.Tensor, ref: np.ndarray, what: str, atomic: bool = True, budget=None) -> float:
     """Backward bar: `atomic` for gradients summed by atomic adds (grad_x),
-    else the tighter bar of gradients reduced in fp32 and stored once."""
+    else the tighter bar of gradients reduced in fp32 and stored once.
+    `budget` (atomic only): the oracle's {"abs_sum", "terms"} for grad_x."""
     g = to_np(gpu)
     nan_g, nan_r = np.isnan(g), np.isnan(ref)
     assert np.array_equal(nan_g, nan_r), f"{what}: NaN pattern differs"
-    g, r = g[~nan_r], ref[~nan_r]
+    keep = ~nan_r
+    g, r = g[keep], ref[keep]
     if r.size == 0:
         return 0.0
     tol = (BWD_TOL if atomic else BWD_TOL_REDUCED)[gpu.dtype]
     rms = float(np.sqrt(np.mean(r * r))) if r.size else 0.0
     bound = tol * (np.abs(r) + rms)
+    if budget is not None:
+        assert atomic, "an error budget applies to atomically summed gradients"
+        C = ref.shape[-1] // budget["terms"].shape[-1]
+        terms = np.repeat(budget["terms"], C, axis=-1)
+        bound = np.maximum(bound, summation_bound(budget["abs_sum"], terms, gpu.dtype)[keep])
     err = np.abs(g - r)
     ratio = err / np.maximum(bound, 1e-300)
     worst = int(np.argmax(ratio))
