@@ -112,6 +112,7 @@ def run_bwd(inp, dev):
     keys = ("feat", "spatial_shape", "scale_start_index", "sampling_location", "weights", "grad_out")
     got = d.deform_agg_backward(*(inp[k].to(dev) for k in keys))
     torch.cuda.synchronize()
+    assert d.lib().dcn_take_device_error() == 0
     ref = oracle.agg_backward(*(inp[k] for k in keys))
     return got, ref
 
@@ -158,3 +159,24 @@ def test_bad_table_rows_are_not_read(cuda_dev):
     ref = oracle.agg_forward(inp["feat"], inp["spatial_shape"], inp["scale_start_index"],
                              inp["sampling_location"], w)
     assert_close_fwd(out, ref, "bad table")
+
+
+def test_backward_clustered_locations(cuda_dev):
+    """Units packed into a few cells of the maps (many reductions into the same
+    feature rows) and a few NaN and far locations."""
+    shape = si.AggShape(B=2, num_cams=3, scales=((18, 40), (9, 20), (4, 10)), num_anchors=60, num_pts=7, G=8,
+                        C=32)
+    inp = si.agg_inputs(shape, 812, with_grad_out=True)
+    rng = np.random.default_rng(813)
+    loc = inp["sampling_location"].numpy()
+    centres = rng.uniform(0.1, 0.9, (5, 2))
+    pick = rng.integers(0, 5, loc.shape[:-1])
+    loc[:] = (centres[pick] + rng.normal(0.0, 0.01, loc.shape)).astype(np.float32)
+    loc[0, 3, 2, 1] = [np.nan, 0.5]
+    loc[1, 10, 0, 2] = [3.0, -2.0]
+    inp["sampling_location"] = torch.from_numpy(loc)
+    (gf, gl, gw), ref = run_bwd(inp, cuda_dev)
+    assert np.isnan(ref["grad_loc"]).sum() == 2
+    assert_close_bwd(gf, ref["grad_feat"], "grad_feat")
+    assert_close_bwd(gw, ref["grad_weights"], "grad_weights", atomic=False)
+    assert_close_bwd(gl, ref["grad_loc"], "grad_loc", atomic=False)
