@@ -10,7 +10,9 @@
 // For 16-bit storage the forward runs one CTA per anchor: its warps split the
 // anchor's (point, camera) pairs, each warp walks the scales of its pairs, and
 // the warps' partial rows are summed through shared memory at the end.  The
-// fp32 forward and the backward are persistent and pair-granular (below).  In
+// fp32 forward and the backward are persistent and pair-granular (below); the
+// fp32 forward decodes each tap once per warp (agg_forward_coop_f32) where
+// the shape allows, else once per lane (agg_forward_pairs_f32).  In
 // the backward each pair belongs to exactly one warp, so the location
 // gradient of a pair is reduced inside the warp and stored without atomics;
 // the weight gradient of (sample, group) is reduced over the lanes of the
