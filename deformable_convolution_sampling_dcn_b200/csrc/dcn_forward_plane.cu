@@ -87,11 +87,11 @@ cudaError_t launch_t(const CoreArgs &a, cudaStream_t stream, bool *handled) {
     s.fd_hw = make_fastdiv((unsigned)(a.Ho * a.Wo));
     s.fd_g = make_fastdiv((unsigned)a.G);
     s.fd_box = make_fastdiv((unsigned)kBoxRows);
-    // One CTA of kStagedMaxThreads per SM: a producer warp stages the bands of
+    // One CTA of staged_threads() per SM: a producer warp stages the bands of
     // consecutive segments while the consumer warps gather.  Two band buffers
     // (the next segment loads while the current one is gathered) when they
     // still hold segments of >= 8 output rows with the full halo, else one.
-    const int threads = kStagedMaxThreads, nc = threads / 32 - 1;
+    const int threads = staged_threads(a.softmax, RB, kmax), nc = threads / 32 - 1;
     const size_t other = (size_t)nc * (kmax * IPW * 28 + IPW * 4) + (size_t)kmax * 8 + 32;
     const long long budget = (long long)dev->smem_optin - (long long)other;
     if (budget <= 0) return cudaSuccess;

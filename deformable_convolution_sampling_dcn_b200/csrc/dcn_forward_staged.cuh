@@ -46,7 +46,14 @@
 namespace dcnb {
 
 constexpr uint64_t kStagedWaitNs = 1000000000ull;  // bounded TMA wait: 1 s
-constexpr int kStagedMaxThreads = 512;  // 256 with two CTAs per SM, 512 with one
+// CTA size, one CTA per SM: 15 consumer warps, or 19 in softmax mode, whose
+// longer record phase (a max, exponentials and a sum over K per item) leaves
+// more latency to hide (DCNv3 P3: 167 -> 161 us; the raw-mode P4 instance
+// loses with 640 threads, 41.8 -> 43.5 us, so it keeps 512).  16-byte groups
+// with K > 9 hold 13 raw taps per lane and would spill at 640.
+__host__ __device__ constexpr int staged_threads(bool softmax, int rb, int kmax) {
+    return softmax && !(rb == 32 && kmax > 9) ? 640 : 512;
+}
 
 struct StagedParams {
     CoreArgs a;
@@ -58,7 +65,7 @@ struct StagedParams {
     int halo;           // margin rows
     int seg_rows;       // output rows per segment at most
     unsigned int *err;  // device error word (bit 0: a TMA wait ran out)
-    int threads;        // CTA size (multiple of 32, <= kStagedMaxThreads)
+    int threads;        // CTA size: staged_threads(softmax, RB, KMAX)
     int nbuf;           // band buffers (1 or 2): segment n uses buffer n % nbuf
     FastDiv fd_wo;      // division by Wo
     FastDiv fd_hw;      // division by Ho * Wo (used when n_items < 2^31)
@@ -152,7 +159,7 @@ template <> struct RawTap<__nv_bfloat16> {
 };
 
 template <typename T, int RB, bool SOFTMAX, int KMAX>
-__global__ void __launch_bounds__(kStagedMaxThreads, 1)
+__global__ void __launch_bounds__(staged_threads(SOFTMAX, RB, KMAX), 1)
     core_forward_staged(const __grid_constant__ CUtensorMap tmap, const StagedParams s) {
     constexpr int V = Storage<T>::kVec;  // elements per 16-byte chunk
     constexpr int V2 = V / 2;            // fp32 pairs per chunk
