@@ -14,15 +14,30 @@
 namespace dcnb {
 namespace {
 
-// One warp per (roi, bin); lane l owns 16-byte channel chunks l, l+32, ...
-// (CPL of them, one channel block of 32*CPL chunks at a time).  The bin
+// One warp per (roi, bin); lane l owns channel chunks l, l+32, ... of
+// 16 * W16 bytes (CPL of them, one channel block of 32*CPL chunks at a time;
+// W16 = 2 reads each chunk with one 32-byte load, sm_100's ld.global.v8, for
+// which L1 returns twice the bytes per clock of 16-byte loads).  The bin
 // geometry is computed by every lane (same values).  For each sample the
 // four corner loads of all the lane's chunks are independent and issued
 // together (an out-of-map corner loads nothing and gets weight zero); the
 // sample loop is unrolled by two to keep more loads in flight.
-template <typename T, int CPL>
+template <int W16> struct Chunk { uint4 h[W16]; };
+
+template <int W16> __device__ __forceinline__ Chunk<W16> ld_chunk(const void *p);
+template <> __device__ __forceinline__ Chunk<1> ld_chunk<1>(const void *p) { return Chunk<1>{{ld_nc16(p)}}; }
+template <> __device__ __forceinline__ Chunk<2> ld_chunk<2>(const void *p) {
+    uint32_t q[8];
+    asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3]), "=r"(q[4]), "=r"(q[5]), "=r"(q[6]), "=r"(q[7])
+                 : "l"(p));
+    return Chunk<2>{{make_uint4(q[0], q[1], q[2], q[3]), make_uint4(q[4], q[5], q[6], q[7])}};
+}
+
+template <typename T, int CPL, int W16>
 __global__ void __launch_bounds__(256) roi_pool_forward_kernel(RoiArgs a) {
-    constexpr int V = Storage<T>::kVec;
+    constexpr int V16 = Storage<T>::kVec;  // elements per 16 bytes
+    constexpr int V = V16 * W16;           // elements per chunk
     const int lane = threadIdx.x & 31;
     // N * PH * PW <= 2^31 (checked on the host): 32-bit index arithmetic
     const unsigned bins = (unsigned)a.N * (unsigned)(a.PH * a.PW);
@@ -76,14 +91,21 @@ __global__ void __launch_bounds__(256) roi_pool_forward_kernel(RoiArgs a) {
 #pragma unroll
                     for (int q = 0; q < CPL; ++q) {
                         if (lane + 32 * q >= left) break;
-                        uint4 raw[4];
+                        Chunk<W16> raw[4];
 #pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            raw[c] = off[c] >= 0 ? ld_nc16(xb + off[c] + 32 * q * V) : make_uint4(0, 0, 0, 0);
+                        for (int c = 0; c < 4; ++c) {
+                            if (off[c] >= 0) {
+                                raw[c] = ld_chunk<W16>(xb + off[c] + 32 * q * V);
+                            } else {
+#pragma unroll
+                                for (int h = 0; h < W16; ++h) raw[c].h[h] = make_uint4(0, 0, 0, 0);
+                            }
+                        }
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
                             float f[V];
-                            unpack16<T>(raw[c], f);
+#pragma unroll
+                            for (int h = 0; h < W16; ++h) unpack16<T>(raw[c].h[h], f + h * V16);
 #pragma unroll
                             for (int v = 0; v < V; ++v) acc[q][v] = fmaf(g[c], f[v], acc[q][v]);
                         }
@@ -98,21 +120,33 @@ __global__ void __launch_bounds__(256) roi_pool_forward_kernel(RoiArgs a) {
             if (c >= left) break;
 #pragma unroll
             for (int v = 0; v < V; ++v) acc[q][v] = nan_pos ? __int_as_float(0x7fc00000) : acc[q][v] * inv;
-            *reinterpret_cast<uint4 *>(o + c * V) = pack16<T>(acc[q]);
+#pragma unroll
+            for (int h = 0; h < W16; ++h)
+                *reinterpret_cast<uint4 *>(o + c * V + h * V16) = pack16<T>(acc[q] + h * V16);
         }
     }
 }
 
-template <typename T>
-cudaError_t launch_t(const RoiArgs &a, cudaStream_t stream) {
+template <typename T, int W16>
+cudaError_t launch_w(const RoiArgs &a, cudaStream_t stream) {
     const long long bins = (long long)a.N * a.PH * a.PW;
     const unsigned blocks = (unsigned)((bins + 7) / 8);
-    const int cpl = (a.C / Storage<T>::kVec + 31) / 32;
-    if (cpl <= 1) roi_pool_forward_kernel<T, 1><<<blocks, 256, 0, stream>>>(a);
-    else if (cpl == 2) roi_pool_forward_kernel<T, 2><<<blocks, 256, 0, stream>>>(a);
-    else if (cpl <= 4) roi_pool_forward_kernel<T, 4><<<blocks, 256, 0, stream>>>(a);
-    else roi_pool_forward_kernel<T, 8><<<blocks, 256, 0, stream>>>(a);
+    const int cpl = (a.C / (Storage<T>::kVec * W16) + 31) / 32;
+    if (cpl <= 1) roi_pool_forward_kernel<T, 1, W16><<<blocks, 256, 0, stream>>>(a);
+    else if (cpl == 2) roi_pool_forward_kernel<T, 2, W16><<<blocks, 256, 0, stream>>>(a);
+    else if (cpl <= 4) roi_pool_forward_kernel<T, 4, W16><<<blocks, 256, 0, stream>>>(a);
+    else roi_pool_forward_kernel<T, 8, W16><<<blocks, 256, 0, stream>>>(a);
     return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_t(const RoiArgs &a, cudaStream_t stream) {
+    // 32-byte chunks where every lane still gets one (rows of at least 1 KB)
+    // and x sits on a 32-byte boundary (rows are then 32-byte multiples too)
+    const long long row = (long long)a.C * sizeof(T);
+    if (row % 32 == 0 && row >= 1024 && (reinterpret_cast<uintptr_t>(a.x) & 31) == 0)
+        return launch_w<T, 2>(a, stream);
+    return launch_w<T, 1>(a, stream);
 }
 
 }  // namespace
