@@ -65,6 +65,9 @@ def _bind(lib):
     lib.oracle_dcn_backward.restype = None
     lib.oracle_dcn_grad_x_budget.argtypes = [i] * 13 + [ctypes.c_float, i, dp, dp, dp, dp, dp]
     lib.oracle_dcn_grad_x_budget.restype = None
+    lib.oracle_agg_grad_feat_budget.argtypes = [i] * 8 + [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int),
+                                                          ctypes.POINTER(ctypes.c_float), dp, dp, dp, dp]
+    lib.oracle_agg_grad_feat_budget.restype = None
     lib.oracle_agg_forward.argtypes = [i] * 8 + [dp, ip, ip, fp, dp, dp]
     lib.oracle_agg_forward.restype = None
     lib.oracle_agg_backward.argtypes = [i] * 8 + [dp, ip, ip, fp, dp, dp, dp, dp, dp]
@@ -247,6 +250,24 @@ def agg_backward(feat, spatial_shape, scale_start_index, sampling_location, weig
                             _ptr(go, ctypes.c_double), _ptr(gf, ctypes.c_double),
                             _ptr(gl, ctypes.c_double), _ptr(gw, ctypes.c_double))
     return {"grad_feat": gf, "grad_loc": gl, "grad_weights": gw}
+
+
+def agg_grad_feat_budget(feat, spatial_shape, scale_start_index, sampling_location, weights, grad_out,
+                         lib=None) -> Dict[str, np.ndarray]:
+    """Per grad_feat element: the absolute sum of its contributions (abs_sum,
+    [B, rows, G*C]) and their number (terms, [B, rows, G]); see dcn_oracle.c."""
+    lib = lib or load()
+    feat, ss, st, loc, w, dims = _agg_common(feat, spatial_shape, scale_start_index,
+                                             sampling_location, weights)
+    B, cams, S, rows, A, P, G, C = dims
+    go = _f64(grad_out)
+    abs_sum = np.empty((B, rows, G * C), dtype=np.float64)
+    terms = np.empty((B, rows, G), dtype=np.float64)
+    lib.oracle_agg_grad_feat_budget(*dims, _ptr(ss, ctypes.c_int), _ptr(st, ctypes.c_int),
+                                    _ptr(loc, ctypes.c_float), _ptr(w, ctypes.c_double),
+                                    _ptr(go, ctypes.c_double), _ptr(abs_sum, ctypes.c_double),
+                                    _ptr(terms, ctypes.c_double))
+    return {"abs_sum": abs_sum, "terms": terms}
 
 
 def roi_pool_forward(x, rois, offset, *, pooled=(7, 7), sampling=2, spatial_scale: float = 1.0,

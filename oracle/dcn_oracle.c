@@ -533,6 +533,56 @@ void oracle_agg_backward(int B, int cams, int S, int rows, int A, int P, int G, 
 }
 
 /*
+ * Error budget of the aggregation's feature gradient, summed by atomic
+ * additions on a device: per grad_feat element the sum of the absolute values
+ * of its contributions |w G(q,p) grad_out_c| (abs_sum, [B, rows, G*C]) and how
+ * many it receives (terms, [B, rows, G]); see oracle_dcn_grad_x_budget for the
+ * bound these give.  The samples are enumerated exactly as in
+ * oracle_agg_backward.
+ */
+void oracle_agg_grad_feat_budget(int B, int cams, int S, int rows, int A, int P, int G, int C,
+                                 const int *shape, const int *start, const float *loc,
+                                 const double *weights, const double *grad_out,
+                                 double *abs_sum, double *terms)
+{
+    memset(abs_sum, 0, sizeof(double) * (size_t)B * rows * G * C);
+    memset(terms, 0, sizeof(double) * (size_t)B * rows * G);
+#pragma omp parallel for collapse(2) schedule(dynamic)
+    for (int b = 0; b < B; ++b)
+        for (int g = 0; g < G; ++g)
+            for (int a = 0; a < A; ++a) {
+                const double *go = grad_out + (((size_t)b * A + a) * G + g) * C;
+                for (int p = 0; p < P; ++p)
+                    for (int cam = 0; cam < cams; ++cam) {
+                        const float *l = loc + ((((size_t)b * A + a) * P + p) * cams + cam) * 2;
+                        for (int s = 0; s < S; ++s) {
+                            const int Hs = shape[(cam * S + s) * 2 + 0];
+                            const int Ws = shape[(cam * S + s) * 2 + 1];
+                            const float px = fmaf(l[0], (float)Ws, -0.5f);
+                            const float py = fmaf(l[1], (float)Hs, -0.5f);
+                            const double w = weights[(((((size_t)b * A + a) * P + p) * cams + cam) * S + s) * G + g];
+                            if (isnan(px) || isnan(py)) continue;
+                            const double fy = floor((double)py), fx = floor((double)px);
+                            if (!(fy >= -1.0 && fy <= Hs - 1 && fx >= -1.0 && fx <= Ws - 1)) continue;
+                            const int y0 = (int)fy, x0 = (int)fx;
+                            for (int qy = y0; qy <= y0 + 1; ++qy) {
+                                if (qy < 0 || qy >= Hs) continue;
+                                for (int qx = x0; qx <= x0 + 1; ++qx) {
+                                    if (qx < 0 || qx >= Ws) continue;
+                                    const double Gq = g_kernel(qx, px) * g_kernel(qy, py);
+                                    const size_t row = (size_t)b * rows + (size_t)start[cam * S + s] +
+                                                       (size_t)qy * Ws + qx;
+                                    double *aq = abs_sum + row * (size_t)G * C + (size_t)g * C;
+                                    for (int c = 0; c < C; ++c) aq[c] += fabs(w * Gq * go[c]);
+                                    terms[row * G + g] += 1.0;
+                                }
+                            }
+                        }
+                    }
+            }
+}
+
+/*
  * Deformable RoI pooling, forward ("用PyTorch实战DCNv1：从零构建可变形卷积与ROI池化模块",
  * section 3): the k x k bins of a region of interest are each moved by a
  * learned offset normalised by the region size, dp = gamma * dp_hat o (w, h),

@@ -443,6 +443,51 @@ def pin_agg_backward(lib):
     assert abs(lhs - rhs) < 1e-10 * (1 + abs(lhs)), "agg adjoint"
 
 
+def pin_agg_grad_feat_budget(lib):
+    """The aggregation's grad_feat budget by brute force over every (anchor,
+    point, camera, scale, group, corner), positions formed in fp32; and, for
+    non-negative weights and grad_out, the absolute sum is grad_feat itself."""
+    for B in (1, 2):
+        feat, shape, start, loc, w = agg_case(420 + B, B=B, quant=2.0 ** -12)
+        rng = np.random.default_rng(430 + B)
+        _, rows, GC = feat.shape
+        _, A, P, cams, S, G = w.shape
+        C = GC // G
+        go = rng.standard_normal((B, A, GC))
+        bud = oracle.agg_grad_feat_budget(feat, shape, start, loc, w, go, lib=lib)
+        absum = np.zeros((B, rows, GC))
+        n = np.zeros((B, rows, G))
+        for b in range(B):
+            for a in range(A):
+                for p in range(P):
+                    for cam in range(cams):
+                        for s in range(S):
+                            Hs, Ws = shape[cam, s]
+                            px = agg_pos32(loc[b, a, p, cam, 0:1], Ws)[0]
+                            py = agg_pos32(loc[b, a, p, cam, 1:2], Hs)[0]
+                            y0, x0 = int(np.floor(py)), int(np.floor(px))
+                            for qy in (y0, y0 + 1):
+                                for qx in (x0, x0 + 1):
+                                    if not (0 <= qy < Hs and 0 <= qx < Ws):
+                                        continue
+                                    wgt = max(0.0, 1 - abs(qx - px)) * max(0.0, 1 - abs(qy - py))
+                                    if wgt == 0.0:
+                                        continue
+                                    row = start[cam, s] + qy * Ws + qx
+                                    for g in range(G):
+                                        sl = slice(g * C, (g + 1) * C)
+                                        absum[b, row, sl] += np.abs(w[b, a, p, cam, s, g] * wgt * go[b, a, sl])
+                                        n[b, row, g] += 1
+        assert np.allclose(bud["abs_sum"], absum, rtol=1e-12, atol=1e-14), "agg abs_sum"
+        assert np.array_equal(bud["terms"], n), "agg terms"
+    feat, shape, start, loc, w = agg_case(440, quant=2.0 ** -12)
+    go = np.abs(np.random.default_rng(441).standard_normal((1, w.shape[1], feat.shape[2])))
+    w = np.abs(w)
+    gr = oracle.agg_backward(feat, shape, start, loc, w, go, lib=lib)
+    bud = oracle.agg_grad_feat_budget(feat, shape, start, loc, w, go, lib=lib)
+    assert np.allclose(bud["abs_sum"], gr["grad_feat"], rtol=1e-12, atol=1e-14), "agg abs_sum vs grad_feat"
+
+
 CORE_PINS = [pin_identity, pin_box_sum, pin_shifted_gather, pin_affine_field, pin_softmax_constant,
              pin_softmax_vs_raw, pin_brute_force]
 def pin_backward_right_derivative_at_minus_one(lib):
@@ -529,7 +574,7 @@ def pin_grad_x_budget(lib):
 
 BACKWARD_PINS = [pin_backward_fd, pin_backward_autograd, pin_backward_right_derivative_at_minus_one,
                  pin_grad_x_budget]
-AGG_PINS = [pin_agg_brute_force, pin_agg_grid_sample, pin_agg_backward]
+AGG_PINS = [pin_agg_brute_force, pin_agg_grid_sample, pin_agg_backward, pin_agg_grad_feat_budget]
 ALL_PINS = CORE_PINS + BACKWARD_PINS + AGG_PINS
 
 

@@ -27,7 +27,8 @@ contributions and n itself), an element may instead stay within the
 recursive-summation bound gamma_(n+1) * A, gamma_m = m u / (1 - m u), u the
 storage type's unit roundoff (2^-24, 2^-11, 2^-8): the bound that holds for
 any order of the atomic additions, which matters where a sum cancels far
-below its terms.
+below its terms.  Where (n+1) u >= 1/2 (over 127 additions in bf16) no
+useful bound exists and the element is checked for its NaN pattern only.
 NaN must match NaN exactly.
 """
 from __future__ import annotations
@@ -75,9 +76,14 @@ UNIT_ROUNDOFF = {torch.float32: 2.0 ** -24, torch.float16: 2.0 ** -11, torch.bfl
 
 def summation_bound(abs_sum: np.ndarray, terms: np.ndarray, dtype: torch.dtype) -> np.ndarray:
     """gamma_(n+1) * A: the error bound of n contributions with absolute sum A
-    added one by one, each partial sum and each contribution rounded once."""
+    added one by one, each partial sum and each contribution rounded once.
+    The bound holds while (n+1) u < 1; where (n+1) u >= 1/2 (more than 127
+    additions in bf16, 1023 in fp16) it exceeds A itself and the element is
+    left unbounded (infinite): a 16-bit running sum of that many terms can lose
+    every significant bit, in any order of the additions."""
     mu = (terms + 1.0) * UNIT_ROUNDOFF[dtype]
-    return mu / (1.0 - mu) * abs_sum
+    with np.errstate(divide="ignore"):
+        return np.where(mu < 0.5, mu / (1.0 - np.minimum(mu, 0.5)) * abs_sum, np.inf)
 
 
 def assert_close_bwd(gpu: torch.Tensor, ref: np.ndarray, what: str, atomic: bool = True, budget=None) -> float:

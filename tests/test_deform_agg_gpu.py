@@ -34,7 +34,7 @@ def test_sparse4d_backward_generic(cuda_dev, monkeypatch):
     shape = si.AggShape(B=1, num_cams=3, scales=((16, 44), (8, 22)), num_anchors=40, num_pts=5, G=8, C=32)
     inp = si.agg_inputs(shape, 77, with_grad_out=True, loc_lo=-0.05, loc_hi=1.05)
     (gf, gl, gw), ref = run_bwd(inp, cuda_dev)
-    assert_close_bwd(gf, ref["grad_feat"], "grad_feat")
+    assert_close_bwd(gf, ref["grad_feat"], "grad_feat", budget=ref["budget"])
     assert_close_bwd(gw, ref["grad_weights"], "grad_weights")
     assert_close_bwd(gl, ref["grad_loc"], "grad_loc")
 
@@ -114,6 +114,7 @@ def run_bwd(inp, dev):
     torch.cuda.synchronize()
     assert d.lib().dcn_take_device_error() == 0
     ref = oracle.agg_backward(*(inp[k] for k in keys))
+    ref["budget"] = oracle.agg_grad_feat_budget(*(inp[k] for k in keys))
     return got, ref
 
 
@@ -122,7 +123,7 @@ def test_small_backward(case, cuda_dev):
     shape, lr = small_shape(case)
     inp = si.agg_inputs(shape, 400 + case, loc_lo=lr[0], loc_hi=lr[1], with_grad_out=True)
     (gf, gl, gw), ref = run_bwd(inp, cuda_dev)
-    assert_close_bwd(gf, ref["grad_feat"], "grad_feat")
+    assert_close_bwd(gf, ref["grad_feat"], "grad_feat", budget=ref["budget"])
     assert_close_bwd(gw, ref["grad_weights"], "grad_weights")
     # locations are fp32 in every dtype; their gradient sums fp32 atomics
     gl64 = gl.double().cpu().numpy()
@@ -135,7 +136,7 @@ def test_small_backward(case, cuda_dev):
 def test_sparse4d_backward_full_size(cuda_dev):
     inp = si.agg_inputs(si.SPARSE4D, si.SEEDS["sparse4d"], with_grad_out=True)
     (gf, gl, gw), ref = run_bwd(inp, cuda_dev)
-    assert_close_bwd(gf, ref["grad_feat"], "grad_feat")
+    assert_close_bwd(gf, ref["grad_feat"], "grad_feat", budget=ref["budget"])
     assert_close_bwd(gw, ref["grad_weights"], "grad_weights")
     assert_close_bwd(gl, ref["grad_loc"], "grad_loc")
 
@@ -177,6 +178,6 @@ def test_backward_clustered_locations(cuda_dev):
     inp["sampling_location"] = torch.from_numpy(loc)
     (gf, gl, gw), ref = run_bwd(inp, cuda_dev)
     assert np.isnan(ref["grad_loc"]).sum() == 2
-    assert_close_bwd(gf, ref["grad_feat"], "grad_feat")
+    assert_close_bwd(gf, ref["grad_feat"], "grad_feat", budget=ref["budget"])
     assert_close_bwd(gw, ref["grad_weights"], "grad_weights", atomic=False)
     assert_close_bwd(gl, ref["grad_loc"], "grad_loc", atomic=False)
