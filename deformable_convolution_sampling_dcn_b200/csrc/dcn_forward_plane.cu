@@ -1,7 +1,7 @@
 // Host-side planning of the staged forward (kernel in dcn_forward_staged.cuh):
-// picks the band height, the halo and one or two CTAs per SM from the shared
-// memory budget, builds the 4-D TMA tensor map of x, and launches the
-// persistent grid.  Shapes the staged kernel does not cover (W > 254,
+// picks the band height, the halo and one or two band buffers from the shared
+// memory budget left by the records of staged_threads() warps, builds the 4-D
+// TMA tensor map of x, and launches the persistent grid of one CTA per SM.  Shapes the staged kernel does not cover (W > 254,
 // K > 25, 16-byte groups, a map the tensor-map encoder rejects) are left to
 // the generic kernel.
 #include <cudaTypedefs.h>
