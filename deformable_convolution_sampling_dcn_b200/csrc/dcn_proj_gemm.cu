@@ -69,6 +69,7 @@ struct GemmParams {
     const void *bias;  // [Cout] or nullptr
     void *out;
     unsigned int *err;
+    int store32;       // out rows start on 32-byte boundaries: 32-byte stores (whole L2 sectors)
 };
 
 template <typename T>
@@ -244,9 +245,21 @@ __global__ void __launch_bounds__(kGThreads, 1)
                 if (row < p.P) {
                     T *dst = out + row * p.Cout + o0;
                     const int n16 = (p.Cout - o0) >= 32 ? 4 : (p.Cout - o0) / 8;  // Cout is a multiple of 8
+                    if (p.store32 && n16 == 4) {
+                        // two 32-byte stores: every store fills whole 32-byte sectors of L2
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        if (i < n16) reinterpret_cast<uint4 *>(dst)[i] = pack16<T>(v + 8 * i);
+                        for (int i = 0; i < 2; ++i) {
+                            const uint4 lo = pack16<T>(v + 16 * i), hi = pack16<T>(v + 16 * i + 8);
+                            asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(dst + 16 * i),
+                                         "r"(lo.x), "r"(lo.y), "r"(lo.z), "r"(lo.w), "r"(hi.x), "r"(hi.y), "r"(hi.z),
+                                         "r"(hi.w)
+                                         : "memory");
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            if (i < n16) reinterpret_cast<uint4 *>(dst)[i] = pack16<T>(v + 8 * i);
+                    }
                 }
             }
             tc_fence_before();
@@ -288,6 +301,7 @@ cudaError_t launch_t(const void *core, const void *weight, const void *bias, voi
     p.bias = bias;
     p.out = out;
     p.err = dev->err;
+    p.store32 = Cout % 16 == 0 && (reinterpret_cast<uintptr_t>(out) & 31) == 0;
 
     CUtensorMap amap, bmap;
     const cuuint32_t estr[2] = {1, 1};
